@@ -1,0 +1,485 @@
+/*
+ * Reference oracle for InstaGen group-shared importance-sampled permuted
+ * block-sparse attention (one DiT self-attention call, per head).
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is a plain, slow, obviously correct CPU
+ * statement of what the GPU path computes.  Only the tests, the smoke check and
+ * the benchmark's CPU-baseline leg may load it; the product path never does.
+ * It shares no code, header, table or constant generator with the CUDA library.
+ *
+ * Sources (web pages on "InstaGen: Group-Shared Importance Sampling for Fast
+ * Video Generation", arXiv 2611.08610):
+ *   [ABS]   the paper's abstract (paper-reading aggregator page and the
+ *           thelatestinai.com paper page): block selection cast as importance
+ *           sampling; top-scoring keys form an exact set computed in full; the
+ *           remaining keys are a sample drawn in proportion to their estimated
+ *           attention and reweighted by inverse sampling probability; one
+ *           sample per query cluster shared by all of its queries.
+ *   [FIG3]  thelatestinai.com paper page, Figure 3 caption: (a) queries and
+ *           keys are clustered into groups; (b) centroid scores give each key
+ *           group a probability pi for each query group; (c) the top key group
+ *           is always kept, the rest are sampled in proportion to pi and
+ *           weighted by 1/pi; (d) queries of a group share keys, so attention
+ *           runs over dense blocks in one kernel.
+ *   [FIG2]  same page, Figure 2 caption: SVG2 clustering configuration
+ *           Cq = 100 query and Ck = 500 key clusters.
+ *   [ICLR]  acceptodds.com ICLR 2027 listing, abstract: the sample is shared
+ *           across all queries of the cluster and computed together with the
+ *           top-k blocks in one attention kernel, sampled scores reweighted
+ *           to stand for the whole skipped region.
+ *
+ * Where the pages are silent the plainest reading is taken; each such reading
+ * is marked "[reading]" below.
+ *
+ * Floating point: everything that decides an integer (scores, ranking, the
+ * integer sampling weights) uses single-precision operations that are
+ * correctly rounded (multiply, add, fmaf, floorf, ldexpf), so any conforming
+ * implementation reaches the same bits.  Build with -ffp-contract=off.
+ * Everything else (distances, means, softmax, log-weights) is fp64.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_OK 0
+#define ORC_ERR_ARG 1
+#define ORC_ERR_NOMEM 2
+
+/* ------------------------------------------------------------------------- */
+/* Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy
+ * as 1, 2, 3", SC 2011).  Round: two 32x32->64 multiplies by the Philox
+ * multipliers, outputs permuted and xored with the key; the key is bumped by
+ * the Weyl constants (golden ratio and sqrt(3)-1 in 32-bit fixed point)
+ * between rounds.  Ten rounds.                                               */
+/* ------------------------------------------------------------------------- */
+void orc_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint32_t out[4])
+{
+    const uint32_t mul0 = 0xD2511F53u, mul1 = 0xCD9E8D57u;
+    const uint32_t weyl0 = 0x9E3779B9u, weyl1 = 0xBB67AE85u;
+    uint32_t c0 = ctr_in[0], c1 = ctr_in[1], c2 = ctr_in[2], c3 = ctr_in[3];
+    uint32_t k0 = key_in[0], k1 = key_in[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) { k0 += weyl0; k1 += weyl1; }
+        uint64_t p0 = (uint64_t)mul0 * (uint64_t)c0;
+        uint64_t p1 = (uint64_t)mul1 * (uint64_t)c2;
+        uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        uint32_t n0 = hi1 ^ c1 ^ k0;
+        uint32_t n1 = lo1;
+        uint32_t n2 = hi0 ^ c3 ^ k1;
+        uint32_t n3 = lo0;
+        c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* Batch form used by the tests: ctrs [n,4], keys [n,2] -> out [n,4]. */
+void orc_philox_batch(int64_t n, const uint32_t* ctrs, const uint32_t* keys, uint32_t* out)
+{
+    for (int64_t i = 0; i < n; ++i) orc_philox4x32_10(ctrs + 4 * i, keys + 2 * i, out + 4 * i);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Budgets.  [reading] E and m are the given shares of the N keys rounded to
+ * the nearest integer, halves away from zero (Table 1 caption of the paper
+ * page: "E + S", exact and sampled share of keys per sparse call).           */
+/* ------------------------------------------------------------------------- */
+int64_t orc_budget(float frac, int64_t N)
+{
+    return (int64_t)llround((double)frac * (double)N);
+}
+
+/* ------------------------------------------------------------------------- */
+/* (a) k-means clustering of one head's queries or keys [FIG3 (a)].
+ * [reading] squared Euclidean distance; initial centroid j is token
+ * floor(j*N/C); ties go to the lowest centroid index; an empty cluster keeps
+ * its previous centroid; T Lloyd iterations of (assign, update), so the
+ * returned centroids are the means of the returned clusters.                */
+/* ------------------------------------------------------------------------- */
+void orc_kmeans_init(const float* X, int64_t N, int d, int C, float* cent)
+{
+    for (int j = 0; j < C; ++j) {
+        int64_t src = ((int64_t)j * N) / C;
+        memcpy(cent + (int64_t)j * d, X + src * d, sizeof(float) * (size_t)d);
+    }
+}
+
+/* assign[i] = argmin_j ||x_i - c_j||^2 in fp64, lowest j on ties.
+ * inertia (optional) = sum_i min_j ||x_i - c_j||^2.                          */
+void orc_kmeans_assign(const float* X, int64_t N, int d, const float* cent, int C,
+                       int32_t* assign, double* inertia)
+{
+    double total = 0.0;
+    #pragma omp parallel for schedule(static) reduction(+:total)
+    for (int64_t i = 0; i < N; ++i) {
+        const float* x = X + i * d;
+        double best = INFINITY;
+        int32_t best_j = 0;
+        for (int j = 0; j < C; ++j) {
+            const float* c = cent + (int64_t)j * d;
+            double dist = 0.0;
+            for (int k = 0; k < d; ++k) {
+                double diff = (double)x[k] - (double)c[k];
+                dist += diff * diff;
+            }
+            if (dist < best) { best = dist; best_j = j; }
+        }
+        assign[i] = best_j;
+        total += best;
+    }
+    if (inertia) *inertia = total;
+}
+
+/* c_j = mean of its members (fp64 sum in ascending token order, rounded to
+ * fp32); an empty cluster keeps its centroid.                               */
+int orc_kmeans_update(const float* X, int64_t N, int d, const int32_t* assign, int C, float* cent)
+{
+    double* sums = (double*)calloc((size_t)C * (size_t)d, sizeof(double));
+    int64_t* counts = (int64_t*)calloc((size_t)C, sizeof(int64_t));
+    if (!sums || !counts) { free(sums); free(counts); return ORC_ERR_NOMEM; }
+    for (int64_t i = 0; i < N; ++i) {
+        int32_t a = assign[i];
+        if (a < 0 || a >= C) { free(sums); free(counts); return ORC_ERR_ARG; }
+        counts[a] += 1;
+        for (int k = 0; k < d; ++k) sums[(int64_t)a * d + k] += (double)X[i * d + k];
+    }
+    for (int j = 0; j < C; ++j) {
+        if (counts[j] == 0) continue;
+        for (int k = 0; k < d; ++k)
+            cent[(int64_t)j * d + k] = (float)(sums[(int64_t)j * d + k] / (double)counts[j]);
+    }
+    free(sums); free(counts);
+    return ORC_OK;
+}
+
+/* Full k-means: init (or the given centroids), then iters x (assign, update).
+ * inertia_hist (optional, length iters) records the inertia of each assign. */
+int orc_kmeans(const float* X, int64_t N, int d, int C, int iters, const float* init,
+               float* cent, int32_t* assign, double* inertia_hist)
+{
+    if (C < 1 || N < 1 || d < 1 || iters < 1) return ORC_ERR_ARG;
+    if (init) memcpy(cent, init, sizeof(float) * (size_t)C * (size_t)d);
+    else orc_kmeans_init(X, N, d, C, cent);
+    for (int t = 0; t < iters; ++t) {
+        double inertia = 0.0;
+        orc_kmeans_assign(X, N, d, cent, C, assign, &inertia);
+        if (inertia_hist) inertia_hist[t] = inertia;
+        int rc = orc_kmeans_update(X, N, d, assign, C, cent);
+        if (rc) return rc;
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Semantic permutation [ABS "semantically permuted attention matrix",
+ * FIG3 (d)].  [reading] stable counting sort by cluster id: cluster j owns
+ * the contiguous range [offsets[j], offsets[j+1]); inside it tokens keep
+ * ascending original index.  perm[p] = original index at permuted slot p.    */
+/* ------------------------------------------------------------------------- */
+int orc_permutation(const int32_t* assign, int64_t N, int C, int32_t* perm, int32_t* offsets)
+{
+    int64_t* cursor = (int64_t*)calloc((size_t)C + 1, sizeof(int64_t));
+    if (!cursor) return ORC_ERR_NOMEM;
+    for (int64_t i = 0; i < N; ++i) {
+        if (assign[i] < 0 || assign[i] >= C) { free(cursor); return ORC_ERR_ARG; }
+        cursor[assign[i] + 1] += 1;
+    }
+    for (int j = 0; j < C; ++j) cursor[j + 1] += cursor[j];
+    for (int j = 0; j <= C; ++j) offsets[j] = (int32_t)cursor[j];
+    for (int64_t i = 0; i < N; ++i) perm[cursor[assign[i]]++] = (int32_t)i;
+    free(cursor);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* (b) Centroid scores [FIG3 (b)].  S_ij = scale * <cq_i, ck_j>.
+ * [reading] the dot product is one fused multiply-add chain in fp32 over
+ * k = 0..d-1 starting from +0, then one fp32 multiply by the softmax scale:
+ * every step correctly rounded, hence reproducible bit for bit.              */
+/* ------------------------------------------------------------------------- */
+void orc_scores(const float* cq, int Cq, const float* ck, int Ck, int d, float scale, float* S)
+{
+    for (int i = 0; i < Cq; ++i)
+        for (int j = 0; j < Ck; ++j) {
+            float acc = 0.0f;
+            for (int k = 0; k < d; ++k)
+                acc = fmaf(cq[(int64_t)i * d + k], ck[(int64_t)j * d + k], acc);
+            S[(int64_t)i * Ck + j] = acc * scale;
+        }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Integer sampling weight of a skipped key group [ABS "drawn in proportion to
+ * their estimated attention"; FIG3 (b),(c)].
+ * [reading] the estimated attention of every key of group j, seen from query
+ * group i, is exp(S_ij); the group's mass is |K_j| exp(S_ij), so a key's
+ * probability is proportional to q_j ~ 2^24 * exp(S_ij - Smax).  It is held
+ * as an integer in [1, 2^24] so that every implementation draws the same
+ * indices; exp is evaluated as 2^y with y = (S_ij - Smax) * log2(e) split into
+ * an integer and a fractional part, and 2^f = e^(f ln 2) by its Taylor series
+ * up to degree 6 (Horner, fmaf).  Keys are never given weight 0 (q >= 1), so
+ * every skipped key stays reachable and 1/pi stays finite.  Unbiasedness only
+ * needs the log-weight to use the q that was sampled from, not an exact exp. */
+/* ------------------------------------------------------------------------- */
+static float orc_taylor_coef[7];
+static int orc_taylor_ready = 0;
+
+static void orc_taylor_init(void)
+{
+    /* coefficient k = (ln 2)^k / k!, computed in fp64 and rounded once. */
+    double term = 1.0;
+    for (int k = 0; k <= 6; ++k) {
+        orc_taylor_coef[k] = (float)term;
+        term = term * M_LN2 / (double)(k + 1);
+    }
+    orc_taylor_ready = 1;
+}
+
+void orc_taylor_coefficients(float* out7)
+{
+    if (!orc_taylor_ready) orc_taylor_init();
+    for (int k = 0; k < 7; ++k) out7[k] = orc_taylor_coef[k];
+}
+
+uint32_t orc_group_weight(float s, float smax)
+{
+    if (!orc_taylor_ready) orc_taylor_init();
+    const float log2e = (float)1.4426950408889634; /* log2(e) rounded to fp32 */
+    float y = (s - smax) * log2e;
+    if (y < -24.0f) return 1u;
+    float n = floorf(y);
+    float f = y - n;
+    float p = orc_taylor_coef[6];
+    for (int k = 5; k >= 0; --k) p = fmaf(p, f, orc_taylor_coef[k]);
+    float v = floorf(ldexpf(p, 24 + (int)n));
+    uint32_t q = (uint32_t)v;
+    return q < 1u ? 1u : q;
+}
+
+/* ------------------------------------------------------------------------- */
+/* (c) Exact set, pi and the group-shared sample for one query group i.
+ *
+ * Exact set [ABS "top-scoring keys form an exact set that is computed in
+ * full"; FIG3 (c) "the top key group is always kept"].  [reading] non-empty
+ * key groups ranked by S_ij descending (ties: lowest j); the rank-0 group is
+ * always taken; the next groups are taken while the running key count stays
+ * <= E, stopping at the first group that does not fit (a prefix of the
+ * ranking).
+ *
+ * Sample [ABS, FIG3 (c), ICLR].  The skipped keys are the keys of the
+ * non-empty groups outside the exact set.  [reading] m draws with replacement,
+ * one shared list per query group; draw t uses Philox4x32-10 with key =
+ * (seed low, seed high) and counter = (t, i, bh, layer); u = r1*2^32 + r0,
+ * r = floor(u * T / 2^64) with T = sum_j |K_j| q_j over skipped groups (j
+ * ascending, the CDF order); the group is the first with CDF_j > r and the
+ * key offset in it is (r - CDF_{j-1}) / q_j (integer division: uniform inside
+ * the group).  The key's probability is p = q_j / T, and its log-weight is
+ * log(1/(p m)) = ln T - ln q_j - ln m, which is added to its logit so that
+ * the m draws stand for the whole skipped region (ICLR "reweighted to account
+ * for the full skipped region").  No skipped keys -> no draws.
+ *
+ * Uniform variant (mode 1; Figure 2/4/5 captions run "uniform" sampling):
+ * q_j = 1 for every skipped group.
+ *
+ * Outputs for the group:
+ *   exact_groups[0..n_exact)  group ids in rank order (rest set to -1)
+ *   counts[0] = n_exact groups, counts[1] = exact keys, counts[2] = draws
+ *   sample_pos[0..draws)      permuted key positions, in draw order
+ *   sample_bias[0..draws)     log-weights (fp64)
+ *   qw[j], cdf info (optional) for the tests
+ * ------------------------------------------------------------------------- */
+typedef struct {
+    int64_t E, m;
+    uint64_t seed;
+    uint32_t layer, bh;
+    int mode; /* 0 importance, 1 uniform */
+} orc_select_cfg;
+
+int orc_select_sample_group(const float* S_row, const int32_t* k_offsets, int Ck, int i,
+                            const orc_select_cfg* cfg,
+                            int32_t* exact_groups, int32_t* counts,
+                            int32_t* sample_pos, double* sample_bias,
+                            uint32_t* qw_out /* [Ck] or NULL: 0 for non-skipped */,
+                            uint64_t* total_out /* or NULL */)
+{
+    int32_t* order = (int32_t*)malloc(sizeof(int32_t) * (size_t)(Ck > 0 ? Ck : 1));
+    uint8_t* in_exact = (uint8_t*)calloc((size_t)(Ck > 0 ? Ck : 1), 1);
+    uint32_t* qw = (uint32_t*)calloc((size_t)(Ck > 0 ? Ck : 1), sizeof(uint32_t));
+    uint64_t* cdf = (uint64_t*)calloc((size_t)(Ck > 0 ? Ck : 1), sizeof(uint64_t));
+    if (!order || !in_exact || !qw || !cdf) { free(order); free(in_exact); free(qw); free(cdf); return ORC_ERR_NOMEM; }
+
+    /* rank the non-empty groups: plain insertion sort, S descending, j ascending */
+    int nz = 0;
+    for (int j = 0; j < Ck; ++j) {
+        if (k_offsets[j + 1] - k_offsets[j] <= 0) continue;
+        int pos = nz++;
+        while (pos > 0) {
+            int prev = order[pos - 1];
+            float sp = S_row[prev], sj = S_row[j];
+            int before = (sp > sj) || (sp == sj && prev < j);
+            if (before) break;
+            order[pos] = prev;
+            --pos;
+        }
+        order[pos] = j;
+    }
+
+    for (int r = 0; r < Ck; ++r) exact_groups[r] = -1;
+    int n_exact = 0;
+    int64_t exact_keys = 0;
+    for (int r = 0; r < nz; ++r) {
+        int j = order[r];
+        int64_t cnt = k_offsets[j + 1] - k_offsets[j];
+        if (r > 0 && exact_keys + cnt > cfg->E) break;
+        exact_groups[n_exact++] = j;
+        in_exact[j] = 1;
+        exact_keys += cnt;
+    }
+
+    /* pi over the skipped groups */
+    int any_skipped = 0;
+    float smax = -INFINITY;
+    for (int j = 0; j < Ck; ++j) {
+        if (in_exact[j] || k_offsets[j + 1] - k_offsets[j] <= 0) continue;
+        if (!any_skipped || S_row[j] > smax) smax = S_row[j];
+        any_skipped = 1;
+    }
+    uint64_t total = 0;
+    for (int j = 0; j < Ck; ++j) {
+        int64_t cnt = k_offsets[j + 1] - k_offsets[j];
+        if (in_exact[j] || cnt <= 0) { cdf[j] = total; continue; }
+        qw[j] = (cfg->mode == 1) ? 1u : orc_group_weight(S_row[j], smax);
+        total += (uint64_t)cnt * (uint64_t)qw[j];
+        cdf[j] = total; /* inclusive */
+    }
+
+    int64_t draws = any_skipped ? cfg->m : 0;
+    const uint32_t key[2] = { (uint32_t)(cfg->seed & 0xffffffffu), (uint32_t)(cfg->seed >> 32) };
+    const double log_total = log((double)total);
+    const double log_m = draws > 0 ? log((double)draws) : 0.0;
+    for (int64_t t = 0; t < draws; ++t) {
+        uint32_t ctr[4] = { (uint32_t)t, (uint32_t)i, cfg->bh, cfg->layer };
+        uint32_t rnd[4];
+        orc_philox4x32_10(ctr, key, rnd);
+        uint64_t u = ((uint64_t)rnd[1] << 32) | (uint64_t)rnd[0];
+        uint64_t r = (uint64_t)(((unsigned __int128)u * (unsigned __int128)total) >> 64);
+        int jsel = -1;
+        for (int j = 0; j < Ck; ++j) {
+            if (in_exact[j] || k_offsets[j + 1] - k_offsets[j] <= 0) continue;
+            if (cdf[j] > r) { jsel = j; break; }
+        }
+        if (jsel < 0) { free(order); free(in_exact); free(qw); free(cdf); return ORC_ERR_ARG; }
+        uint64_t start = cdf[jsel] - (uint64_t)(k_offsets[jsel + 1] - k_offsets[jsel]) * qw[jsel];
+        uint64_t o = (r - start) / qw[jsel];
+        sample_pos[t] = k_offsets[jsel] + (int32_t)o;
+        sample_bias[t] = log_total - log((double)qw[jsel]) - log_m;
+    }
+
+    counts[0] = n_exact;
+    counts[1] = (int32_t)exact_keys;
+    counts[2] = (int32_t)draws;
+    if (qw_out) memcpy(qw_out, qw, sizeof(uint32_t) * (size_t)Ck);
+    if (total_out) *total_out = total;
+    free(order); free(in_exact); free(qw); free(cdf);
+    return ORC_OK;
+}
+
+/* Whole head: scores from the given centroids, then every query group.
+ * exact_groups [Cq,Ck], counts [Cq,3], sample_pos [Cq,m], sample_bias [Cq,m].
+ * Unused sample slots hold position -1 and log-weight 0.                      */
+int orc_select_sample(const float* cq, int Cq, const float* ck, int Ck, int d, float scale,
+                      const int32_t* k_offsets, const orc_select_cfg* cfg,
+                      int32_t* exact_groups, int32_t* counts,
+                      int32_t* sample_pos, double* sample_bias)
+{
+    float* S = (float*)malloc(sizeof(float) * (size_t)Cq * (size_t)Ck);
+    if (!S) return ORC_ERR_NOMEM;
+    orc_scores(cq, Cq, ck, Ck, d, scale, S);
+    int rc = ORC_OK;
+    for (int i = 0; i < Cq && rc == ORC_OK; ++i) {
+        int32_t* sp = sample_pos + (int64_t)i * cfg->m;
+        double* sb = sample_bias + (int64_t)i * cfg->m;
+        for (int64_t t = 0; t < cfg->m; ++t) { sp[t] = -1; sb[t] = 0.0; }
+        rc = orc_select_sample_group(S + (int64_t)i * Ck, k_offsets, Ck, i, cfg,
+                                     exact_groups + (int64_t)i * Ck, counts + 3 * i,
+                                     sp, sb, NULL, NULL);
+    }
+    free(S);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------- */
+/* (d) Attention over the exact keys plus the weighted sample [ABS, FIG3 (d),
+ * ICLR].  For query q (original index) in group i = q_assign[q]:
+ *   keys   = every key of the exact groups (original index k_perm[p] for p in
+ *            [k_off[g], k_off[g+1])) and every sample slot t (original index
+ *            k_perm[sample_pos[i][t]]), a key drawn twice counting twice;
+ *   logit  = scale * <q, k>  (+ sample_bias[i][t] for slot t);
+ *   out    = sum softmax(logit) * v, all in fp64.
+ * rows lists the original query indices to compute; out is [nrows, d].      */
+/* ------------------------------------------------------------------------- */
+int orc_attention_rows(const float* Q, const float* K, const float* V, int64_t N, int d, float scale,
+                       const int32_t* q_assign, const int32_t* k_perm, const int32_t* k_offsets, int Ck,
+                       const int32_t* exact_groups, const int32_t* counts,
+                       const int32_t* sample_pos, const double* sample_bias, int64_t m_stride,
+                       const int64_t* rows, int64_t nrows, double* out)
+{
+    int bad = 0;
+    #pragma omp parallel for schedule(dynamic, 4) reduction(|:bad)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t q = rows[r];
+        double* o = out + r * d;
+        for (int k = 0; k < d; ++k) o[k] = 0.0;
+        if (q < 0 || q >= N) { bad |= 1; continue; }
+        int i = q_assign[q];
+        const float* qv = Q + q * d;
+        int ne = counts[3 * i + 0], ns = counts[3 * i + 2];
+        /* pass 1: maximum logit */
+        double mx = -INFINITY;
+        for (int e = 0; e < ne; ++e) {
+            int g = exact_groups[(int64_t)i * Ck + e];
+            for (int32_t p = k_offsets[g]; p < k_offsets[g + 1]; ++p) {
+                const float* kv = K + (int64_t)k_perm[p] * d;
+                double s = 0.0;
+                for (int k = 0; k < d; ++k) s += (double)qv[k] * (double)kv[k];
+                s *= (double)scale;
+                if (s > mx) mx = s;
+            }
+        }
+        for (int t = 0; t < ns; ++t) {
+            int32_t p = sample_pos[(int64_t)i * m_stride + t];
+            const float* kv = K + (int64_t)k_perm[p] * d;
+            double s = 0.0;
+            for (int k = 0; k < d; ++k) s += (double)qv[k] * (double)kv[k];
+            s = s * (double)scale + sample_bias[(int64_t)i * m_stride + t];
+            if (s > mx) mx = s;
+        }
+        /* pass 2: weights and the weighted sum of values */
+        double den = 0.0;
+        for (int e = 0; e < ne; ++e) {
+            int g = exact_groups[(int64_t)i * Ck + e];
+            for (int32_t p = k_offsets[g]; p < k_offsets[g + 1]; ++p) {
+                int64_t kk = k_perm[p];
+                const float* kv = K + kk * d;
+                double s = 0.0;
+                for (int k = 0; k < d; ++k) s += (double)qv[k] * (double)kv[k];
+                double w = exp(s * (double)scale - mx);
+                den += w;
+                for (int k = 0; k < d; ++k) o[k] += w * (double)V[kk * d + k];
+            }
+        }
+        for (int t = 0; t < ns; ++t) {
+            int32_t p = sample_pos[(int64_t)i * m_stride + t];
+            int64_t kk = k_perm[p];
+            const float* kv = K + kk * d;
+            double s = 0.0;
+            for (int k = 0; k < d; ++k) s += (double)qv[k] * (double)kv[k];
+            double w = exp(s * (double)scale + sample_bias[(int64_t)i * m_stride + t] - mx);
+            den += w;
+            for (int k = 0; k < d; ++k) o[k] += w * (double)V[kk * d + k];
+        }
+        for (int k = 0; k < d; ++k) o[k] /= den;
+    }
+    return bad ? ORC_ERR_ARG : ORC_OK;
+}
