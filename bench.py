@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of one InstaGen attention call (cluster Q and K, permute/gather,
+select + group-shared sample, sparse attention) on B200.
+
+Metric: ms per attention call (lower is better), plus effective TFLOP/s on the
+attended FLOPs (sum over heads and query groups of 4 * n_i * (exact_i + m) * d)
+as a fraction of the measured bf16 tensor-core peak.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   (the CPU oracle, bounded sample)
+
+Multi-GPU: the call does not shard across GPUs (one call per GPU); N ranks run
+N independent calls (replicas, one layer each), no collective on the data
+path; value = aggregate ms per call = max-over-ranks time / (K * N).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="instagen", choices=["instagen", "reference"])
+    ap.add_argument("--workload", default="wan2.1-14b_720p")
+    ap.add_argument("--exact", type=float, default=None, help="override the exact share")
+    ap.add_argument("--sample", type=float, default=None, help="override the sampled share")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sust=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, source="fallback")
+
+
+def attention_traffic_per_unit():
+    """DRAM bytes per attended key-row (from the committed ncu summary) if it was
+    captured on the current attention kernel source, else None."""
+    path = os.path.join(ROOT, "profiles", "attention_traffic.json")
+    src = os.path.join(ROOT, "block_sparse_attention_head_b200", "csrc", "attention.cu")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    with open(src, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()
+    if d.get("attention_cu_sha256") != h:
+        return None
+    return d
+
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"instagen_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={SMI_FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx, "samples": len(mhz),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------- CPU oracle
+class OracleSample:
+    """The CPU oracle on a bounded sample of the workload (one head).
+
+    Set-up (untimed): the head's inputs and one oracle k-means iteration (its
+    centroids and lists feed the timed stages).  One timed step: k-means
+    assign + update of 4096 sampled tokens against the Q and K centroids
+    (x N/4096 tokens, x iters), select/sample of the head's query groups, and
+    attention for 32 query rows (x N/32); extrapolated x B*H heads.
+    """
+
+    def __init__(self, w, exact, sample, seed=0):
+        import numpy as np
+        import oracle
+        from block_sparse_attention_head_b200 import workloads
+        oracle.build()
+        self.np, self.oracle, self.w = np, oracle, w
+        Q, K, V = workloads.make_inputs(w, heads=[0])
+        self.Q, self.K, self.V = (t[0, 0].float().numpy() for t in (Q, K, V))
+        self.scale = 1.0 / math.sqrt(w.d)
+        self.cq, self.qa, _ = oracle.kmeans(self.Q, w.Cq, 1)
+        self.ck, self.ka, _ = oracle.kmeans(self.K, w.Ck, 1)
+        self.kp, self.ko = oracle.permutation(self.ka, w.Ck)
+        self.E, self.m = oracle.budget(exact, w.N), oracle.budget(sample, w.N)
+        self.seed = seed
+        self.rng = np.random.default_rng(0)
+        self.n_tok, self.n_rows = min(4096, w.N), min(32, w.N)
+
+    def step(self):
+        o, w, np = self.oracle, self.w, self.np
+        tok = self.rng.choice(w.N, self.n_tok, replace=False)
+        t0 = time.perf_counter()
+        for X, cent in ((self.Q, self.cq), (self.K, self.ck)):
+            xs = np.ascontiguousarray(X[tok])
+            a, _ = o.kmeans_assign(xs, cent)
+            o.kmeans_update(xs, a, cent)
+        t_km = time.perf_counter() - t0
+        t1 = time.perf_counter()
+        ex, cnt, sp, sb = o.select_sample(self.cq, self.ck, self.ko, self.scale, self.E, self.m, seed=self.seed)
+        t_sel = time.perf_counter() - t1
+        rows = self.rng.choice(w.N, self.n_rows, replace=False)
+        t2 = time.perf_counter()
+        o.attention_rows(self.Q, self.K, self.V, self.scale, self.qa, self.kp, self.ko, ex, cnt, sp, sb, rows)
+        t_att = time.perf_counter() - t2
+        per_head = t_km * (w.N / self.n_tok) * w.iters + t_sel + t_att * (w.N / self.n_rows)
+        return per_head * w.B * w.H * 1e3
+
+    def describe(self):
+        w = self.w
+        return (f"head 0 of {w.name}: k-means assign+update of {self.n_tok} tokens for Q and K "
+                f"(x{w.N / self.n_tok:.1f} tokens, x{w.iters} iterations), select/sample of the head, "
+                f"attention on {self.n_rows} query rows (x{w.N / self.n_rows:.0f}); extrapolated x{w.B * w.H} heads")
+
+
+def reference_arm(args, w, exact, sample):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    t0 = time.perf_counter()
+    orc = OracleSample(w, exact, sample)
+    for _ in range(args.warmup):
+        orc.step()
+    vals = [orc.step() for _ in range(args.steps)]
+    ms = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": "ms per InstaGen attention call", "value": round(ms, 1),
+        "unit": "ms/call", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, exact, sample),
+        "cpu_baseline": {"kind": "oracle", "cores": orc.oracle.num_threads(), "sample": orc.describe(),
+                         "value": round(ms, 1), "unit": "ms/call"},
+        "e2e": {"value": round(ms, 1), "unit": "ms/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": round(time.perf_counter() - t0, 1),
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def workload_config(w, exact, sample):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "Cq": w.Cq, "Ck": w.Ck,
+            "kmeans_iters": w.iters, "exact_frac": exact, "sample_frac": sample, "sampling": "importance",
+            "inputs": "clustered Gaussian mixture (seeded), bf16",
+            "l2": "inputs (Q,K,V %.1f GB per call) larger than L2" % (3 * w.B * w.H * w.N * w.d * 2 / 1e9)}
+
+
+# ------------------------------------------------------------------ GPU arm
+def main():
+    args = parse_args()
+    from block_sparse_attention_head_b200 import workloads
+    w = workloads.WORKLOADS[args.workload]
+    exact = w.exact_frac if args.exact is None else args.exact
+    sample = w.sample_frac if args.sample is None else args.sample
+    if args.impl == "reference":
+        return reference_arm(args, w, exact, sample)
+
+    import torch
+    import block_sparse_attention_head_b200 as ig
+    from block_sparse_attention_head_b200 import build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    build.build()
+    ig.lib()
+
+    peaks = load_peaks()
+    dev = torch.device("cuda", local)
+    Q, K, V = workloads.make_inputs(w, layer=rank, device=dev)
+    p = ig.make_params(w.B, w.H, w.N, w.d, w.Cq, w.Ck, iters=w.iters, exact_frac=exact, sample_frac=sample,
+                       seed=1000 + rank, layer=rank)
+    ws = torch.empty(ig.workspace_size(p), dtype=torch.uint8, device=dev)
+    O = torch.empty_like(Q)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---------------- headline: instagen_forward, inputs resident in HBM
+    for _ in range(args.warmup):
+        ig.forward(Q, K, V, p, workspace=ws, out=O)
+    ig.device_status()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            ig.forward(Q, K, V, p, workspace=ws, out=O)
+        ev1.record(stream)
+        barrier()
+    ig.device_status()
+    t_fwd = ev0.elapsed_time(ev1)
+    clocks = clk.summary()
+
+    # ---------------- stage breakdown: the same calls, staged, with events
+    inter = ig.forward_intermediates(ws, p)
+    stages = ["cluster_q", "cluster_k", "gather_kv", "select_sample", "attention"]
+    acc = {s: 0.0 for s in stages}
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+    barrier()
+    for _ in range(args.steps):
+        evs[0].record(stream)
+        cq, qa, qp, qo = ig.cluster(Q, w.Cq, w.iters, p)
+        evs[1].record(stream)
+        ck, ka, kp, ko = ig.cluster(K, w.Ck, w.iters, p)
+        evs[2].record(stream)
+        Kp, Vp = ig.gather(K, kp, p), ig.gather(V, kp, p)
+        evs[3].record(stream)
+        eg, cnt, sp, sb = ig.select_sample(cq, ck, ko, p)
+        evs[4].record(stream)
+        ig.attention(Q, Kp, Vp, qp, qo, ko, eg, cnt, sp, sb, p, out=O)
+        evs[5].record(stream)
+        torch.cuda.synchronize()
+        for i, s in enumerate(stages):
+            acc[s] += evs[i].elapsed_time(evs[i + 1])
+        del cq, qa, qp, qo, ck, ka, kp, ko, Kp, Vp, eg, cnt, sp, sb
+    ig.device_status()
+    stage_ms = {s: acc[s] / args.steps for s in stages}
+
+    # ---------------- algorithmic work (from the call's own lists)
+    counts = inter["counts"].long().cpu()
+    qoff = inter["q_offsets"].long().cpu()
+    n_i = (qoff[..., 1:] - qoff[..., :-1])
+    keys_i = counts[..., 1] + counts[..., 2]
+    attended_flops = float((4 * n_i * keys_i * w.d).sum())
+    attended_rows = float((n_i * keys_i).sum())          # (query, key) pairs
+    key_tile_loads = float((((n_i + 127) // 128) * keys_i).sum())  # K/V rows streamed per query tile
+    density = attended_rows / (w.B * w.H * w.N * w.N)
+    t_att = stage_ms["attention"]
+    achieved = attended_flops / (t_att * 1e-3) / 1e12
+    # HBM-side stages: algorithmic bytes
+    BH, N, d = w.B * w.H, w.N, w.d
+    m = ig.sample_budget(p)
+    bytes_cluster = lambda C: w.iters * (BH * N * d * 2 * 2 + BH * N * 4 * 3) + BH * C * d * 4 * 2
+    hbm = {
+        "cluster_q": bytes_cluster(w.Cq), "cluster_k": bytes_cluster(w.Ck),
+        "gather_kv": 2 * 2 * BH * N * d * 2 + BH * N * 4,
+        "select_sample": BH * w.Cq * (m * 8 + w.Ck * 4) + BH * (w.Cq + w.Ck) * d * 4,
+    }
+    stage_report = {}
+    for s in stages:
+        e = {"ms": round(stage_ms[s], 3)}
+        if s in hbm:
+            gbs = hbm[s] / (stage_ms[s] * 1e-3) / 1e9
+            e.update(gbs=round(gbs, 1), hbm_frac=round(gbs / peaks["hbm"], 3))
+        stage_report[s] = e
+    kmeans_flops = 2 * BH * N * (w.Cq + w.Ck) * d * 2 * w.iters     # hi+lo operand: K = 2d
+    stage_report["cluster_q"]["tensor_tflops"] = round(
+        2 * BH * N * w.Cq * d * 2 * w.iters / (stage_ms["cluster_q"] * 1e-3) / 1e12, 1)
+    stage_report["cluster_k"]["tensor_tflops"] = round(
+        2 * BH * N * w.Ck * d * 2 * w.iters / (stage_ms["cluster_k"] * 1e-3) / 1e12, 1)
+
+    traffic = None
+    tr = attention_traffic_per_unit()
+    if tr is not None and tr.get("workload") == w.name and abs(tr.get("exact_frac", -1) - exact) < 1e-9 \
+            and abs(tr.get("sample_frac", -1) - sample) < 1e-9:
+        traffic = tr["dram_bytes_per_launch"]
+
+    # ---------------- dense comparator (torch SDPA) and error vs dense
+    extra = {}
+    if not args.no_dense:
+        import torch.nn.functional as F
+        for _ in range(2):
+            D = F.scaled_dot_product_attention(Q, K, V, scale=p.softmax_scale)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(3):
+            D = F.scaled_dot_product_attention(Q, K, V, scale=p.softmax_scale)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        extra["dense_sdpa_ms"] = round(e0.elapsed_time(e1) / 3, 3)
+        ig.forward(Q, K, V, p, workspace=ws, out=O)
+        num = (O.float() - D.float()).pow(2).sum().sqrt()
+        den = D.float().pow(2).sum().sqrt()
+        extra["rel_l2_vs_dense"] = round(float(num / den), 4)
+        del D
+
+    # ---------------- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
+        hO = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+        dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+
+        def e2e_step():
+            dQ.copy_(hQ, non_blocking=True)
+            dK.copy_(hK, non_blocking=True)
+            dV.copy_(hV, non_blocking=True)
+            ig.forward(dQ, dK, dV, p, workspace=ws, out=O)
+            hO.copy_(O, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        ksteps = max(1, min(args.steps, 5))
+        for _ in range(ksteps):
+            e2e_step()
+        a1.record(stream)
+        barrier()
+        t_e2e = a0.elapsed_time(a1) / ksteps
+        e2e = {"value": t_e2e, "unit": "ms/call", "h2d_bytes_per_step": 3 * Q.numel() * 2,
+               "d2h_bytes_per_step": O.numel() * 2, "steps": ksteps}
+        del hQ, hK, hV, hO, dQ, dK, dV
+
+    # ---------------- max over ranks
+    t_max = t_fwd
+    if dist is not None:
+        tt = torch.tensor([t_fwd, e2e["value"] if e2e else 0.0], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt[0])
+        if e2e:
+            e2e["value"] = float(tt[1])
+    ms_call = t_max / args.steps
+    value = ms_call / world
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        orc = OracleSample(w, exact, sample)
+        orc.step()
+        vals = [orc.step() for _ in range(3)]
+        cpu = {"value": round(statistics.median(vals), 1), "unit": "ms/call", "cores": orc.oracle.num_threads(),
+               "kind": "oracle", "sample": orc.describe() + "; median of 3 steps"}
+
+    launches_per_step = 2 * (1 + 3 * w.iters) + 1 + 1 + 1
+    peak_sust = peaks["bf16_sust"]
+    line = {
+        "metric": "ms per InstaGen attention call", "value": round(value, 3), "unit": "ms/call",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_call, 3),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, exact, sample),
+        "effective_tflops": round(attended_flops / (ms_call * 1e-3) / 1e12, 1),
+        "attended_flops": attended_flops, "density": round(density, 4),
+        "roofline": {"kernel": "attention", "bound": "tensor", "achieved": round(achieved, 1),
+                     "peak": peak_sust, "unit": "TFLOP/s", "frac": round(achieved / peak_sust, 4),
+                     "peak_kind": f"bf16 sustained ({peaks['source']})",
+                     "frac_of_burst": round(achieved / peaks["bf16"], 4),
+                     "traffic": traffic, "algorithmic_unit": "4*d FLOPs per attended (query,key) pair",
+                     "ms": round(t_att, 3)},
+        "stages": stage_report,
+        "e2e": ({"value": round(e2e["value"], 3), "unit": "ms/call", "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
+                 "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]} if e2e else None),
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+        **extra,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,343 @@
+// C ABI of libinstagen.so (declared in include/instagen.h): argument checks,
+// workspace carving, TMA descriptor setup and the launch sequence of the
+// InstaGen attention call (cluster -> permute/gather -> select/sample ->
+// attend).  Nothing here computes on the host beyond shapes and budgets.
+#include "instagen.h"
+#include "internal.cuh"
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+namespace {
+
+using ig::KmeansGeom;
+
+inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape and parameter checks shared by every entry point.
+int check_params(const instagen_params* p) {
+  if (!p) return IG_ERR_INVALID_ARG;
+  if (p->B < 1 || p->H < 1 || p->N < 1) return IG_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return IG_ERR_UNSUPPORTED;
+  const long long bh = (long long)p->B * p->H;
+  if (bh > 65535) return IG_ERR_UNSUPPORTED;                       // grid.y
+  if (bh * (long long)p->N > 2147483647LL - 1024) return IG_ERR_UNSUPPORTED;  // int32 row indices
+  if (!std::isfinite(p->exact_frac) || !std::isfinite(p->sample_frac) || p->exact_frac < 0.f ||
+      p->sample_frac < 0.f)
+    return IG_ERR_INVALID_ARG;
+  if (!std::isfinite(p->softmax_scale)) return IG_ERR_INVALID_ARG;
+  if (p->sampling != IG_SAMPLE_IMPORTANCE && p->sampling != IG_SAMPLE_UNIFORM) return IG_ERR_INVALID_ARG;
+  return IG_OK;
+}
+
+int check_clusters(int C) {
+  if (C < 1) return IG_ERR_INVALID_ARG;
+  if (C > 4096) return IG_ERR_UNSUPPORTED;
+  return IG_OK;
+}
+
+long long budget(float frac, int N) { return (long long)llround((double)frac * (double)N); }
+
+int check_budgets(const instagen_params* p) {
+  const long long m = budget(p->sample_frac, p->N);
+  const long long E = budget(p->exact_frac, p->N);
+  if (m > 2147483647LL || E > 2147483647LL) return IG_ERR_UNSUPPORTED;
+  if ((long long)p->B * p->H * p->Cq * (m > 0 ? m : 1) > (1LL << 40)) return IG_ERR_UNSUPPORTED;
+  return IG_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? IG_OK : IG_ERR_CUDA; }
+
+// ------------------------------------------------------------ TMA descriptors
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// 2-D bf16 row-major [rows, cols] tensor, box {64 columns, box_rows rows},
+// 128-byte swizzle (the UMMA K-major SWIZZLE_128B layout), zero fill outside.
+int make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return IG_ERR_CUDA;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? IG_OK : IG_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- cluster
+int run_cluster(const void* X, int C, int iters, const float* init, const instagen_params* p, float* cent,
+                int32_t* assign, int32_t* perm, int32_t* offsets, void* ws, size_t ws_bytes, cudaStream_t s) {
+  const int BH = p->B * p->H;
+  const KmeansGeom g = ig::kmeans_geom(BH, p->N, p->d, C);
+  if (!ws || ws_bytes < ig::kmeans_scratch_bytes(g) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return IG_ERR_WORKSPACE;
+  __nv_bfloat16* cmma = static_cast<__nv_bfloat16*>(ws);
+  float* norms = reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                          align256((size_t)BH * g.c_pad * 2 * g.d * sizeof(__nv_bfloat16)));
+  CUtensorMap tx, tc;
+  int rc = make_tmap_bf16(&tx, X, (uint64_t)BH * p->N, (uint64_t)p->d, 128);
+  if (rc) return rc;
+  rc = make_tmap_bf16(&tc, cmma, (uint64_t)BH * g.c_pad, (uint64_t)2 * p->d, (uint32_t)g.chunk);
+  if (rc) return rc;
+  const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
+  cudaError_t e = ig::launch_kmeans_init(g, Xb, init, cent, cmma, norms, s);
+  for (int it = 0; it < iters && e == cudaSuccess; ++it) {
+    e = ig::launch_kmeans_assign(g, &tx, &tc, norms, assign, s);
+    if (e == cudaSuccess) e = ig::launch_count_sort(assign, BH, p->N, C, perm, offsets, s);
+    if (e == cudaSuccess) e = ig::launch_kmeans_update(g, Xb, perm, offsets, cent, cmma, norms, s);
+  }
+  return cuda_status(e);
+}
+
+struct ForwardLayout {
+  instagen_forward_layout l;
+};
+
+int forward_layout(const instagen_params* p, instagen_forward_layout* L) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if ((rc = check_clusters(p->Cq)) || (rc = check_clusters(p->Ck))) return rc;
+  if ((rc = check_budgets(p))) return rc;
+  const size_t BH = (size_t)p->B * p->H, N = p->N, d = p->d;
+  const size_t m = (size_t)budget(p->sample_frac, p->N);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  L->cq = take(BH * p->Cq * d * 4);
+  L->ck = take(BH * p->Ck * d * 4);
+  L->q_assign = take(BH * N * 4);
+  L->k_assign = take(BH * N * 4);
+  L->q_perm = take(BH * N * 4);
+  L->k_perm = take(BH * N * 4);
+  L->q_offsets = take(BH * (p->Cq + 1) * 4);
+  L->k_offsets = take(BH * (p->Ck + 1) * 4);
+  L->kp = take(BH * N * d * 2);
+  L->vp = take(BH * N * d * 2);
+  L->exact_groups = take(BH * p->Cq * p->Ck * 4);
+  L->counts = take(BH * p->Cq * 3 * 4);
+  L->sample_pos = take(BH * p->Cq * (m ? m : 1) * 4);
+  L->sample_bias = take(BH * p->Cq * (m ? m : 1) * 4);
+  const size_t cq_ws = ig::kmeans_scratch_bytes(ig::kmeans_geom((int)BH, p->N, p->d, p->Cq));
+  const size_t ck_ws = ig::kmeans_scratch_bytes(ig::kmeans_geom((int)BH, p->N, p->d, p->Ck));
+  L->cluster_ws = take(cq_ws > ck_ws ? cq_ws : ck_ws);
+  L->total = off;
+  return IG_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t instagen_exact_budget(const instagen_params* p) {
+  if (check_params(p)) return -1;
+  return budget(p->exact_frac, p->N);
+}
+
+int64_t instagen_sample_budget(const instagen_params* p) {
+  if (check_params(p)) return -1;
+  return budget(p->sample_frac, p->N);
+}
+
+const char* instagen_error_string(int status) {
+  switch (status) {
+    case IG_OK: return "ok";
+    case IG_ERR_INVALID_ARG: return "invalid argument";
+    case IG_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+    case IG_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case IG_ERR_CUDA: return "CUDA runtime error";
+    case IG_ERR_DEVICE_CHECK: return "device check failed (index out of range or wait timeout)";
+    default: return "unknown status";
+  }
+}
+
+int instagen_device_status(void* stream) {
+  int v = 0;
+  cudaError_t e = ig::read_and_clear_device_error(&v, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return IG_ERR_CUDA;
+  return v ? IG_ERR_DEVICE_CHECK : IG_OK;
+}
+
+size_t instagen_cluster_workspace_size(const instagen_params* p, int32_t C) {
+  if (check_params(p) || check_clusters(C)) return 0;
+  return ig::kmeans_scratch_bytes(ig::kmeans_geom(p->B * p->H, p->N, p->d, C));
+}
+
+size_t instagen_workspace_size(const instagen_params* p) {
+  instagen_forward_layout L;
+  if (forward_layout(p, &L)) return 0;
+  return L.total;
+}
+
+int instagen_forward_layout_get(const instagen_params* p, instagen_forward_layout* out) {
+  if (!out) return IG_ERR_INVALID_ARG;
+  return forward_layout(p, out);
+}
+
+int instagen_cluster(const void* X, int32_t C, int32_t iters, const float* init, const instagen_params* p,
+                     float* centroids, int32_t* assign, int32_t* perm, int32_t* offsets, void* ws,
+                     size_t ws_bytes, void* stream) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if ((rc = check_clusters(C))) return rc;
+  if (iters < 1 || iters > 10000) return IG_ERR_INVALID_ARG;
+  if (!X || !centroids || !assign || !perm || !offsets || !aligned16(X)) return IG_ERR_INVALID_ARG;
+  return run_cluster(X, C, iters, init, p, centroids, assign, perm, offsets, ws, ws_bytes,
+                     static_cast<cudaStream_t>(stream));
+}
+
+int instagen_permutation(const int32_t* assign, int32_t C, const instagen_params* p, int32_t* perm,
+                         int32_t* offsets, void* stream) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if ((rc = check_clusters(C))) return rc;
+  if (!assign || !perm || !offsets) return IG_ERR_INVALID_ARG;
+  return cuda_status(
+      ig::launch_count_sort(assign, p->B * p->H, p->N, C, perm, offsets, static_cast<cudaStream_t>(stream)));
+}
+
+int instagen_gather(const void* X, const int32_t* perm, const instagen_params* p, void* Xp, void* stream) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if (!X || !perm || !Xp || X == Xp || !aligned16(X) || !aligned16(Xp)) return IG_ERR_INVALID_ARG;
+  return cuda_status(ig::launch_gather_rows(static_cast<const __nv_bfloat16*>(X), nullptr, perm, p->B * p->H,
+                                            p->N, p->d, static_cast<__nv_bfloat16*>(Xp), nullptr,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+int instagen_select_sample(const float* cq, const float* ck, const int32_t* k_offsets, const instagen_params* p,
+                           int32_t* exact_groups, int32_t* counts, int32_t* sample_pos, float* sample_bias,
+                           void* stream) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if ((rc = check_clusters(p->Cq)) || (rc = check_clusters(p->Ck))) return rc;
+  if ((rc = check_budgets(p))) return rc;
+  const long long m = budget(p->sample_frac, p->N);
+  if (!cq || !ck || !k_offsets || !exact_groups || !counts) return IG_ERR_INVALID_ARG;
+  if (m > 0 && (!sample_pos || !sample_bias)) return IG_ERR_INVALID_ARG;
+  ig::SelectArgs a;
+  a.cq = cq;
+  a.ck = ck;
+  a.k_offsets = k_offsets;
+  a.BH = p->B * p->H;
+  a.Cq = p->Cq;
+  a.Ck = p->Ck;
+  a.d = p->d;
+  a.scale = p->softmax_scale;
+  a.E = budget(p->exact_frac, p->N);
+  a.m = m;
+  a.seed = p->seed;
+  a.layer = p->layer;
+  a.mode = p->sampling;
+  a.exact_groups = exact_groups;
+  a.counts = counts;
+  a.sample_pos = sample_pos;
+  a.sample_bias = sample_bias;
+  return cuda_status(ig::launch_select_sample(a, static_cast<cudaStream_t>(stream)));
+}
+
+int instagen_attention(const void* Q, const void* Kp, const void* Vp, const int32_t* q_perm,
+                       const int32_t* q_offsets, const int32_t* k_offsets, const int32_t* exact_groups,
+                       const int32_t* counts, const int32_t* sample_pos, const float* sample_bias,
+                       const instagen_params* p, void* O, void* stream) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if ((rc = check_clusters(p->Cq)) || (rc = check_clusters(p->Ck))) return rc;
+  if (p->Ck > ig::kAttnMaxExactGroups) return IG_ERR_UNSUPPORTED;
+  if ((rc = check_budgets(p))) return rc;
+  const long long m = budget(p->sample_frac, p->N);
+  if (!Q || !Kp || !Vp || !q_perm || !q_offsets || !k_offsets || !exact_groups || !counts || !O)
+    return IG_ERR_INVALID_ARG;
+  if (m > 0 && (!sample_pos || !sample_bias)) return IG_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(Kp) || !aligned16(Vp) || !aligned16(O)) return IG_ERR_INVALID_ARG;
+  ig::AttnArgs a;
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
+  a.Kp = static_cast<const __nv_bfloat16*>(Kp);
+  a.Vp = static_cast<const __nv_bfloat16*>(Vp);
+  a.q_perm = q_perm;
+  a.q_offsets = q_offsets;
+  a.k_offsets = k_offsets;
+  a.exact_groups = exact_groups;
+  a.counts = counts;
+  a.sample_pos = sample_pos;
+  a.sample_bias = sample_bias;
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.BH = p->B * p->H;
+  a.N = p->N;
+  a.d = p->d;
+  a.Cq = p->Cq;
+  a.Ck = p->Ck;
+  a.m = m;
+  a.scale_log2 = p->softmax_scale * 1.4426950408889634f;
+  return cuda_status(ig::launch_attention(a, static_cast<cudaStream_t>(stream)));
+}
+
+int instagen_forward(const void* Q, const void* K, const void* V, void* O, const instagen_params* p, void* ws,
+                     size_t ws_bytes, void* stream) {
+  instagen_forward_layout L;
+  int rc = forward_layout(p, &L);
+  if (rc) return rc;
+  if (p->Ck > ig::kAttnMaxExactGroups) return IG_ERR_UNSUPPORTED;
+  if (p->kmeans_iters < 1 || p->kmeans_iters > 10000) return IG_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return IG_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return IG_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  float* cq = reinterpret_cast<float*>(w + L.cq);
+  float* ck = reinterpret_cast<float*>(w + L.ck);
+  int32_t* qa = reinterpret_cast<int32_t*>(w + L.q_assign);
+  int32_t* ka = reinterpret_cast<int32_t*>(w + L.k_assign);
+  int32_t* qp = reinterpret_cast<int32_t*>(w + L.q_perm);
+  int32_t* kp = reinterpret_cast<int32_t*>(w + L.k_perm);
+  int32_t* qo = reinterpret_cast<int32_t*>(w + L.q_offsets);
+  int32_t* ko = reinterpret_cast<int32_t*>(w + L.k_offsets);
+  void* Kp = w + L.kp;
+  void* Vp = w + L.vp;
+  int32_t* eg = reinterpret_cast<int32_t*>(w + L.exact_groups);
+  int32_t* cnt = reinterpret_cast<int32_t*>(w + L.counts);
+  int32_t* sp = reinterpret_cast<int32_t*>(w + L.sample_pos);
+  float* sb = reinterpret_cast<float*>(w + L.sample_bias);
+  void* cws = w + L.cluster_ws;
+  const size_t cws_bytes = L.total - L.cluster_ws;
+  rc = run_cluster(Q, p->Cq, p->kmeans_iters, nullptr, p, cq, qa, qp, qo, cws, cws_bytes, s);
+  if (rc) return rc;
+  rc = run_cluster(K, p->Ck, p->kmeans_iters, nullptr, p, ck, ka, kp, ko, cws, cws_bytes, s);
+  if (rc) return rc;
+  rc = cuda_status(ig::launch_gather_rows(static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V),
+                                          kp, p->B * p->H, p->N, p->d, static_cast<__nv_bfloat16*>(Kp),
+                                          static_cast<__nv_bfloat16*>(Vp), s));
+  if (rc) return rc;
+  rc = instagen_select_sample(cq, ck, ko, p, eg, cnt, sp, sb, stream);
+  if (rc) return rc;
+  return instagen_attention(Q, Kp, Vp, qp, qo, ko, eg, cnt, sp, sb, p, O, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,78 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace ig {
+
+// ----------------------------------------------------------------- k-means
+// Operand layout of the centroids for the tensor-core distance GEMM:
+// [BH, c_pad, 2d] bf16, columns [0,d) = bf16(c) ("hi"), [d,2d) =
+// bf16(c - hi) ("lo"); norms [BH, c_pad] fp32 = ||c||^2 of the fp32 centroid.
+struct KmeansGeom {
+  int BH, N, d, C;
+  int chunk;   // centroids per MMA chunk (multiple of 16, <= 128)
+  int c_pad;   // C rounded up to a multiple of chunk
+};
+KmeansGeom kmeans_geom(int BH, int N, int d, int C);
+size_t kmeans_scratch_bytes(const KmeansGeom& g);
+
+cudaError_t launch_kmeans_init(const KmeansGeom& g, const __nv_bfloat16* X, const float* init, float* cent,
+                               __nv_bfloat16* cmma, float* norms, cudaStream_t s);
+cudaError_t launch_kmeans_assign(const KmeansGeom& g, const CUtensorMap* tmap_x, const CUtensorMap* tmap_c,
+                                 const float* norms, int32_t* assign, cudaStream_t s);
+cudaError_t launch_kmeans_update(const KmeansGeom& g, const __nv_bfloat16* X, const int32_t* perm,
+                                 const int32_t* offsets, float* cent, __nv_bfloat16* cmma, float* norms,
+                                 cudaStream_t s);
+
+// ------------------------------------------------------- permutation/gather
+cudaError_t launch_count_sort(const int32_t* assign, int BH, int N, int C, int32_t* perm, int32_t* offsets,
+                              cudaStream_t s);
+// Up to two tensors gathered with the same permutation (X1 may be null).
+cudaError_t launch_gather_rows(const __nv_bfloat16* X0, const __nv_bfloat16* X1, const int32_t* perm, int BH,
+                               int N, int d, __nv_bfloat16* Y0, __nv_bfloat16* Y1, cudaStream_t s);
+
+// ---------------------------------------------------------- select/sample
+struct SelectArgs {
+  const float* cq;
+  const float* ck;
+  const int32_t* k_offsets;
+  int BH, Cq, Ck, d;
+  float scale;
+  long long E, m;
+  unsigned long long seed;
+  unsigned layer;
+  int mode;
+  int32_t* exact_groups;
+  int32_t* counts;
+  int32_t* sample_pos;
+  float* sample_bias;
+};
+cudaError_t launch_select_sample(const SelectArgs& a, cudaStream_t s);
+
+// --------------------------------------------------------------- attention
+struct AttnArgs {
+  const __nv_bfloat16* Q;
+  const __nv_bfloat16* Kp;
+  const __nv_bfloat16* Vp;
+  const int32_t* q_perm;
+  const int32_t* q_offsets;
+  const int32_t* k_offsets;
+  const int32_t* exact_groups;
+  const int32_t* counts;
+  const int32_t* sample_pos;
+  const float* sample_bias;
+  __nv_bfloat16* O;
+  int BH, N, d, Cq, Ck;
+  long long m;
+  float scale_log2;  // softmax_scale * log2(e)
+};
+constexpr int kAttnMaxExactGroups = 2048;
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
+
+// ------------------------------------------------------------------ errors
+cudaError_t read_and_clear_device_error(int* value, cudaStream_t s);
+
+}  // namespace ig

@@ -1,0 +1,7 @@
+// Single translation unit of libinstagen.so (the kernels share one device
+// error word, so they are compiled together without relocatable device code).
+#include "permute.cu"
+#include "kmeans.cu"
+#include "select.cu"
+#include "attention.cu"
+#include "api.cu"

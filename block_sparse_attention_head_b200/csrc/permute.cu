@@ -1,0 +1,152 @@
+// Semantic permutation (InstaGen abstract: "a semantically permuted attention
+// matrix"; Figure 3 (d): "queries in a group share the same keys, so attention
+// runs over dense blocks").  A stable counting sort puts every cluster in a
+// contiguous range of slots, and a row gather copies K and V into that order
+// with 128-bit coalesced loads and stores.
+#include "internal.cuh"
+#include "ptx.cuh"
+
+#include <cuda_bf16.h>
+
+namespace ig {
+
+// --------------------------------------------------------- counting sort
+// One CTA per head.  Warp w owns a contiguous segment of the tokens; phase 1
+// counts its segment per cluster, phase 2 turns the (cluster-major,
+// warp-minor) counts into write cursors, phase 3 walks each segment in order
+// (32 tokens at a time, ranks inside a step from __match_any_sync) so equal
+// clusters keep ascending token index.
+__global__ void count_sort_kernel(const int32_t* __restrict__ assign, int N, int C, int32_t* __restrict__ perm,
+                                  int32_t* __restrict__ offsets) {
+  extern __shared__ int cnt[];  // [nwarps][C] counters, then C+1 cluster offsets
+  const int nwarps = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;
+  const int32_t* a = assign + (size_t)bh * N;
+  int* base = cnt + nwarps * C;
+  for (int i = threadIdx.x; i < nwarps * C; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  const int seg = (N + nwarps - 1) / nwarps;
+  const int s0 = min(N, warp * seg), s1 = min(N, s0 + seg);
+  for (int i = s0 + lane; i < s1; i += 32) {
+    const int c = a[i];
+    if (c >= 0 && c < C)
+      atomicAdd(&cnt[warp * C + c], 1);
+    else
+      raise_error(kErrIndex);
+  }
+  __syncthreads();
+  // cluster totals and their exclusive prefix (one warp, sequential over chunks of 32)
+  if (warp == 0) {
+    int run = 0;
+    for (int c0 = 0; c0 < C; c0 += 32) {
+      const int c = c0 + lane;
+      int tot = 0;
+      if (c < C)
+        for (int w = 0; w < nwarps; ++w) tot += cnt[w * C + c];
+      int incl = tot;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (c < C) base[c] = run + incl - tot;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) base[C] = run;
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c <= C; c += blockDim.x) offsets[(size_t)bh * (C + 1) + c] = base[c];
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    int run = base[c];
+    for (int w = 0; w < nwarps; ++w) {
+      const int t = cnt[w * C + c];
+      cnt[w * C + c] = run;
+      run += t;
+    }
+  }
+  __syncthreads();
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int i0 = s0; i0 < s1; i0 += 32) {
+    const int i = i0 + lane;
+    int c = (i < s1) ? a[i] : -1;
+    if (c >= C) c = -1;
+    const unsigned same = __match_any_sync(0xffffffffu, c);
+    const int rank = __popc(same & lt_mask);
+    int pos = 0;
+    if (c >= 0) pos = cnt[warp * C + c] + rank;
+    __syncwarp();
+    if (c >= 0 && rank == 0) cnt[warp * C + c] += __popc(same);
+    __syncwarp();
+    if (c >= 0) perm[(size_t)bh * N + pos] = i;
+  }
+}
+
+cudaError_t launch_count_sort(const int32_t* assign, int BH, int N, int C, int32_t* perm, int32_t* offsets,
+                              cudaStream_t s) {
+  // as many warps (<= 32) as fit 160 KB of per-warp counters
+  int nwarps = (int)((160 * 1024) / ((size_t)C * 4));
+  nwarps = nwarps < 1 ? 1 : (nwarps > 32 ? 32 : nwarps);
+  const size_t sm = ((size_t)nwarps * C + C + 1) * sizeof(int);
+  cudaError_t e = cudaFuncSetAttribute(count_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  count_sort_kernel<<<BH, nwarps * 32, sm, s>>>(assign, N, C, perm, offsets);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- gather
+// Y[bh, p, :] = X[bh, perm[bh, p], :] for one or two tensors; each thread moves
+// 16 bytes, consecutive threads move consecutive chunks of a row.
+__global__ void gather_rows_kernel(const uint4* __restrict__ X0, const uint4* __restrict__ X1,
+                                   const int32_t* __restrict__ perm, long long rows, int N, int cpr,
+                                   uint4* __restrict__ Y0, uint4* __restrict__ Y1) {
+  const long long total = rows * cpr;
+  for (long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x; g < total;
+       g += (long long)gridDim.x * blockDim.x) {
+    const long long row = g / cpr;
+    const int ch = (int)(g - row * cpr);
+    const long long bh = row / N;
+    const int src = perm[row];
+    if (src < 0 || src >= N) {
+      raise_error(kErrIndex);
+      continue;
+    }
+    const long long si = (bh * N + src) * cpr + ch;
+    Y0[g] = X0[si];
+    if (X1) Y1[g] = X1[si];
+  }
+}
+
+cudaError_t launch_gather_rows(const __nv_bfloat16* X0, const __nv_bfloat16* X1, const int32_t* perm, int BH,
+                               int N, int d, __nv_bfloat16* Y0, __nv_bfloat16* Y1, cudaStream_t s) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int cpr = d * 2 / 16;
+  const long long rows = (long long)BH * N;
+  const long long work = rows * cpr;
+  const int threads = 512;
+  long long blocks = (work + threads - 1) / threads;
+  const long long cap = (long long)sms * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  gather_rows_kernel<<<(unsigned)blocks, threads, 0, s>>>(
+      reinterpret_cast<const uint4*>(X0), reinterpret_cast<const uint4*>(X1), perm, rows, N, cpr,
+      reinterpret_cast<uint4*>(Y0), reinterpret_cast<uint4*>(Y1));
+  return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_device_error(int* value, cudaStream_t s) {
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return e;
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  }
+  *value = v;
+  return e;
+}
+
+}  // namespace ig

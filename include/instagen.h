@@ -1,0 +1,206 @@
+/*
+ * instagen.h -- C ABI of libinstagen.so: InstaGen group-shared importance-
+ * sampled permuted block-sparse attention (PBSA) for one DiT self-attention
+ * call, on one NVIDIA B200 (sm_100a).
+ *
+ * Method (InstaGen: Group-Shared Importance Sampling for Fast Video
+ * Generation, arXiv 2611.08610; abstract, and Figure 3 (a)-(d) of the
+ * thelatestinai.com paper page).  Per head:
+ *   (a) queries and keys are clustered into Cq and Ck groups (k-means) and
+ *       permuted so that every group is a contiguous block;
+ *   (b) centroid scores give each query group a probability pi over the key
+ *       groups;
+ *   (c) the top-scoring key groups form an exact set (the top group is always
+ *       kept); the remaining keys are covered by m draws in proportion to pi,
+ *       one list shared by every query of the group, each draw carrying the
+ *       log-weight log(1/(pi*m));
+ *   (d) exact blocks and sampled keys go through one online-softmax kernel.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are contiguous, row-major, on the current CUDA device.
+ *     Q, K, V, O: [B, H, N, d] bf16.  B and H are folded: head bh = b*H + h.
+ *   - Device pointers unless stated.  The caller owns every buffer; the
+ *     library never allocates, frees or synchronises (except
+ *     instagen_device_status, which synchronises the given stream).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
+ *     All work is enqueued asynchronously on it.
+ *   - Return value: an instagen_status.  Argument errors are detected on the
+ *     host before anything is enqueued.  Kernels never trap: an index found
+ *     out of range on the device is skipped and recorded, and a wait that
+ *     exceeds its bound aborts the kernel; both are reported by
+ *     instagen_device_status.
+ *   - Permuted order: cluster c of a head occupies permuted slots
+ *     [offsets[c], offsets[c+1]); perm[p] is the original token index at slot
+ *     p.  Inside a cluster tokens keep ascending original index.
+ */
+#ifndef INSTAGEN_H
+#define INSTAGEN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  IG_OK = 0,
+  IG_ERR_INVALID_ARG = 1,   /* bad pointer, shape, or parameter value            */
+  IG_ERR_UNSUPPORTED = 2,   /* valid but not built (e.g. d not in {64, 128})     */
+  IG_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required        */
+  IG_ERR_CUDA = 4,          /* a CUDA runtime call failed                         */
+  IG_ERR_DEVICE_CHECK = 5   /* a kernel recorded an out-of-range index / timeout */
+} instagen_status;
+
+typedef enum { IG_SAMPLE_IMPORTANCE = 0, IG_SAMPLE_UNIFORM = 1 } instagen_sampling;
+
+typedef struct {
+  int32_t B, H, N, d;        /* shapes; d in {64, 128}; N >= 1                     */
+  int32_t Cq, Ck;            /* query / key cluster counts (Figure 2: 100 / 500)    */
+  int32_t kmeans_iters;      /* Lloyd iterations (>= 1; 10 in every configuration) */
+  float exact_frac;          /* exact share of keys: E = round(exact_frac * N)      */
+  float sample_frac;         /* sampled share: m = round(sample_frac * N) draws      */
+  float softmax_scale;       /* logit scale, usually 1/sqrt(d)                       */
+  uint64_t seed;             /* Philox key                                           */
+  uint32_t layer;            /* Philox counter word 3 (one stream per layer)         */
+  int32_t sampling;          /* instagen_sampling                                    */
+} instagen_params;
+
+/* E and m for these parameters: the share times N rounded to nearest, halves
+ * away from zero (Table 1 caption: "E + S", the exact and sampled shares of
+ * keys per sparse call). */
+int64_t instagen_exact_budget(const instagen_params* p);
+int64_t instagen_sample_budget(const instagen_params* p);
+
+/* Workspace bytes instagen_forward needs for these parameters (0 if invalid).
+ * Other entry points document their own needs. */
+size_t instagen_workspace_size(const instagen_params* p);
+
+/* Workspace bytes instagen_cluster needs for C clusters. */
+size_t instagen_cluster_workspace_size(const instagen_params* p, int32_t C);
+
+/* Human-readable text for a status code (static storage). */
+const char* instagen_error_string(int status);
+
+/* Synchronises `stream`, then returns IG_ERR_DEVICE_CHECK and clears the
+ * device error word if any kernel of this library recorded an out-of-range
+ * index or a wait timeout since the last call; IG_OK otherwise. */
+int instagen_device_status(void* stream);
+
+/*
+ * (a) k-means clustering + stable permutation of one tensor X (Q or K),
+ *     Figure 3 (a); "semantically permuted attention matrix" (abstract).
+ *   X         [B,H,N,d] bf16.
+ *   C         cluster count, 1 <= C <= 4096.
+ *   iters     Lloyd iterations >= 1 (each: assign to the nearest centroid by
+ *             squared Euclidean distance, lowest index on ties; then every
+ *             non-empty cluster's centroid becomes its members' mean, an empty
+ *             cluster keeps its centroid).
+ *   init      [B,H,C,d] fp32 initial centroids, or NULL for centroid j =
+ *             token floor(j*N/C) of the head.
+ *   centroids [B,H,C,d] fp32 out: centroids after the last update (the means
+ *             of the returned clusters).
+ *   assign    [B,H,N] int32 out: cluster of every token (last iteration).
+ *   perm      [B,H,N] int32 out; offsets [B,H,C+1] int32 out (see above).
+ *   ws        >= instagen_cluster_workspace_size(p, C) bytes, 256-B aligned.
+ * Distances are evaluated on the tensor cores as ||c||^2 - 2 x.c with the fp32
+ * centroid split into two bf16 halves (hi + lo) and fp32 accumulation.
+ */
+int instagen_cluster(const void* X, int32_t C, int32_t iters, const float* init, const instagen_params* p,
+                     float* centroids, int32_t* assign, int32_t* perm, int32_t* offsets, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/*
+ * Stable counting sort of given assignments (the permutation step alone).
+ *   assign [B,H,N] int32 in [0, C); perm [B,H,N] out; offsets [B,H,C+1] out.
+ * Out-of-range assignments are an IG_ERR_DEVICE_CHECK (the token is dropped).
+ */
+int instagen_permutation(const int32_t* assign, int32_t C, const instagen_params* p, int32_t* perm,
+                         int32_t* offsets, void* stream);
+
+/*
+ * Gather rows into permuted order: Xp[bh, s, :] = X[bh, perm[bh, s], :].
+ *   X, Xp [B,H,N,d] bf16 (distinct buffers); perm [B,H,N] int32.
+ */
+int instagen_gather(const void* X, const int32_t* perm, const instagen_params* p, void* Xp, void* stream);
+
+/*
+ * (b)+(c) Centroid scores, exact set and the group-shared sample
+ *   (abstract: "top-scoring keys form an exact set that is computed in full
+ *   and the remaining keys are represented by a sample drawn in proportion to
+ *   their estimated attention and reweighted by inverse sampling
+ *   probability"; Figure 3 (b), (c)).
+ *   cq [B,H,Cq,d] fp32, ck [B,H,Ck,d] fp32 centroids; k_offsets [B,H,Ck+1].
+ *   Score S_ij = fp32 fused-multiply-add chain of cq_i . ck_j over k = 0..d-1,
+ *   then one fp32 multiply by softmax_scale (bit-reproducible).
+ *   Exact set of query group i: non-empty key groups ranked by S_ij descending
+ *   (ties: lower j first); rank 0 always; then while the key count stays <= E.
+ *   pi: key k of skipped group j has probability q_j / T, q_j in [1, 2^24] the
+ *   integer 2^24 * exp(S_ij - max skipped S) (uniform mode: q_j = 1), T = sum
+ *   over skipped groups of |K_j| q_j.  Draw t of group i: Philox4x32-10 with
+ *   key (seed low, seed high) and counter (t, i, bh, layer); u = r1*2^32 + r0;
+ *   r = floor(u*T / 2^64); group = first j (ascending) whose inclusive CDF
+ *   exceeds r; key = offsets[j] + (r - CDF_{j-1}) / q_j.  Log-weight
+ *   ln T - ln q_j - ln m (fp32).  No skipped keys: no draws.
+ * Outputs (per head, per query group i):
+ *   exact_groups [B,H,Cq,Ck] int32: exact groups in rank order, then -1.
+ *   counts       [B,H,Cq,3] int32: {exact groups, exact keys, draws}.
+ *   sample_pos   [B,H,Cq,m] int32: permuted key slots in draw order (-1 unused).
+ *   sample_bias  [B,H,Cq,m] fp32 log-weights (0 unused).
+ *   m = instagen_sample_budget(p); sample_pos/sample_bias may be NULL if m = 0.
+ *   Requires Ck <= 4096.
+ */
+int instagen_select_sample(const float* cq, const float* ck, const int32_t* k_offsets, const instagen_params* p,
+                           int32_t* exact_groups, int32_t* counts, int32_t* sample_pos, float* sample_bias,
+                           void* stream);
+
+/*
+ * (d) Sparse attention over exact blocks plus the weighted sample, one
+ *   online-softmax pass (Figure 3 (d); "computes them together with the top-k
+ *   blocks in a single attention kernel", ICLR listing abstract).
+ *   Q  [B,H,N,d] bf16 in ORIGINAL token order (rows gathered via q_perm).
+ *   Kp, Vp [B,H,N,d] bf16 in key-cluster (permuted) order (instagen_gather).
+ *   q_perm, q_offsets: query permutation; k_offsets: key cluster ranges.
+ *   exact_groups, counts, sample_pos, sample_bias: as instagen_select_sample.
+ *   O  [B,H,N,d] bf16 out, ORIGINAL token order.  Query q of group i gets
+ *   softmax over {scale*q.k : k in exact groups of i} U {scale*q.k_t + bias_t :
+ *   sample slots t of i} applied to the matching V rows (a key drawn twice
+ *   counts twice).
+ * QK^T and PV run on the tcgen05 tensor cores (bf16 in, fp32 accumulate in
+ * TMEM); P is rounded to bf16 for the PV product.
+ */
+int instagen_attention(const void* Q, const void* Kp, const void* Vp, const int32_t* q_perm,
+                       const int32_t* q_offsets, const int32_t* k_offsets, const int32_t* exact_groups,
+                       const int32_t* counts, const int32_t* sample_pos, const float* sample_bias,
+                       const instagen_params* p, void* O, void* stream);
+
+/*
+ * The whole call: cluster Q (Cq) and K (Ck), gather K and V into key-cluster
+ * order, select and sample, attend.  O [B,H,N,d] bf16 in original order.
+ * ws >= instagen_workspace_size(p) bytes, 256-B aligned; it holds every
+ * intermediate (layout: instagen_forward_layout).
+ */
+int instagen_forward(const void* Q, const void* K, const void* V, void* O, const instagen_params* p, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/* Byte offsets of instagen_forward's intermediates inside its workspace, so a
+ * caller can inspect them after a call (every offset is 256-B aligned). */
+typedef struct {
+  size_t cq, ck;                 /* fp32 centroids [B,H,Cq,d], [B,H,Ck,d]      */
+  size_t q_assign, k_assign;     /* int32 [B,H,N]                               */
+  size_t q_perm, k_perm;         /* int32 [B,H,N]                               */
+  size_t q_offsets, k_offsets;   /* int32 [B,H,Cq+1], [B,H,Ck+1]                */
+  size_t kp, vp;                 /* bf16 [B,H,N,d] permuted K and V             */
+  size_t exact_groups, counts;   /* int32 [B,H,Cq,Ck], [B,H,Cq,3]               */
+  size_t sample_pos, sample_bias;/* int32 / fp32 [B,H,Cq,m]                     */
+  size_t cluster_ws;             /* scratch for instagen_cluster                */
+  size_t total;                  /* == instagen_workspace_size                  */
+} instagen_forward_layout;
+
+int instagen_forward_layout_get(const instagen_params* p, instagen_forward_layout* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INSTAGEN_H */

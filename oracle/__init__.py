@@ -80,6 +80,7 @@ def _load():
     lib.orc_attention_rows.argtypes = [P, P, P, i64, i32, f32, P, P, P, i32, P, P, P, P, i64,
                                        P, i64, P]
     lib.orc_attention_rows.restype = i32
+    lib.orc_num_threads.restype = i32
     _lib = lib
     return lib
 
@@ -100,6 +101,11 @@ def _i32(a) -> np.ndarray:
 def _check(rc: int, what: str):
     if rc != 0:
         raise RuntimeError(f"oracle {what} failed with code {rc}")
+
+
+def num_threads() -> int:
+    """Threads the oracle's OpenMP loops use."""
+    return int(_load().orc_num_threads())
 
 
 # --------------------------------------------------------------------------- RNG

@@ -483,3 +483,16 @@ int orc_attention_rows(const float* Q, const float* K, const float* V, int64_t N
     }
     return bad ? ORC_ERR_ARG : ORC_OK;
 }
+
+/* Threads an OpenMP parallel region of the oracle uses (for reporting). */
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+int orc_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

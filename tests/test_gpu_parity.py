@@ -1,0 +1,323 @@
+"""GPU parity: every CUDA stage against the CPU oracle on the same seeded
+inputs, through the C ABI.
+
+Inputs flow one way only: seeded generator -> oracle -> (its centroids,
+assignments, permutations, lists) -> the CUDA stage under test.  Nothing the
+CUDA path computes is ever fed to the oracle.
+
+Bars (from the method's statement of parity): indices (permutations, offsets,
+exact sets, sample positions, counts) bit-exact; k-means assignments from the
+same centroids agree on >= 99.9% of tokens; attention output within max-abs
+1e-2 and mean relative error (sum|diff| / sum|ref|) 2e-3 of the fp64 oracle
+on the same bf16 inputs.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_head_b200 as ig
+from block_sparse_attention_head_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 1e-2
+MEAN_REL = 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from block_sparse_attention_head_b200 import build
+    build.build()
+    ig.lib()
+    yield
+    ig.device_status()
+
+
+def np_(t):
+    return t.detach().cpu().numpy()
+
+
+def cuda(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype is not None:
+        t = t.to(dtype)
+    return t.cuda()
+
+
+CASES = {
+    # name: (H, N, d, Cq, Ck, iters, exact, sample, mode, seed)
+    "tiny": (1, 4096, 64, 16, 64, 10, 0.08, 0.08, 0, 0),
+    "ragged_d128": (2, 1000, 128, 7, 40, 4, 0.2, 0.1, 0, 3),
+    "cq1_d64": (1, 777, 64, 1, 13, 3, 0.3, 0.05, 0, 5),
+    "uniform": (1, 2048, 128, 9, 33, 3, 0.1, 0.2, 1, 7),
+    "no_sample": (1, 1500, 64, 6, 20, 3, 0.25, 0.0, 0, 9),
+    "exact_all": (1, 640, 128, 4, 10, 3, 1.0, 0.1, 0, 11),
+    "exact_zero": (1, 900, 64, 5, 30, 3, 0.0, 0.15, 0, 13),
+}
+
+
+def _inputs(case):
+    H, N, d, Cq, Ck, iters, ef, sf, mode, seed = CASES[case]
+    if case == "tiny":
+        Q, K, V = workloads.make_inputs(workloads.TINY)
+    else:
+        Q, K, V = workloads.random_small(seed, N, d, n_centres=12, sigma=0.4, H=H)
+    p = ig.make_params(1, H, N, d, Cq, Ck, iters=iters, exact_frac=ef, sample_frac=sf, seed=1234 + seed,
+                       layer=seed, sampling=mode)
+    return p, Q, K, V
+
+
+def _oracle_head(oracle_mod, p, Q, K, V, h, rows=None):
+    f = lambda t: np_(t[0, h].float())
+    return oracle_mod.forward_head(f(Q), f(K), f(V), Cq=p.Cq, Ck=p.Ck, iters=p.kmeans_iters,
+                                   exact_frac=p.exact_frac, sample_frac=p.sample_frac, scale=p.softmax_scale,
+                                   seed=p.seed, layer=p.layer, bh=h, mode=p.sampling, rows=rows)
+
+
+@pytest.fixture(scope="module")
+def oracle_runs(oracle_mod):
+    out = {}
+    for case in CASES:
+        p, Q, K, V = _inputs(case)
+        out[case] = (p, Q, K, V, [_oracle_head(oracle_mod, p, Q, K, V, h) for h in range(p.H)])
+    return out
+
+
+def _stack(heads, attr, dtype=None):
+    a = np.stack([getattr(h, attr) for h in heads])[None]
+    return cuda(a, dtype)
+
+
+# ------------------------------------------------------------- permutation
+@pytest.mark.parametrize("case", list(CASES))
+def test_permutation_bit_exact(oracle_runs, case):
+    p, Q, K, V, heads = oracle_runs[case]
+    for which, C in (("q", p.Cq), ("k", p.Ck)):
+        assign = _stack(heads, f"{which}_assign")
+        perm, offs = ig.permutation(assign, C, p)
+        assert np.array_equal(np_(perm)[0], np.stack([getattr(h, f"{which}_perm") for h in heads]))
+        assert np.array_equal(np_(offs)[0], np.stack([getattr(h, f"{which}_offsets") for h in heads]))
+    ig.device_status()
+
+
+def test_permutation_edge_cases():
+    # all tokens in one cluster, clusters left empty, single token
+    for N, C, fill in ((333, 5, "one"), (1000, 64, "random"), (1, 3, "one")):
+        p = ig.make_params(1, 1, N, 64, C, C)
+        a = np.full(N, 2 % C, np.int32) if fill == "one" else np.random.default_rng(N).integers(0, C // 2, N)
+        perm, offs = ig.permutation(cuda(a.astype(np.int32)[None, None]), C, p)
+        assert np.array_equal(np_(perm)[0, 0], np.argsort(a, kind="stable"))
+        assert np.array_equal(np_(offs)[0, 0], np.concatenate([[0], np.cumsum(np.bincount(a, minlength=C))]))
+    ig.device_status()
+
+
+# ------------------------------------------------------------------- gather
+@pytest.mark.parametrize("case", ["tiny", "ragged_d128"])
+def test_gather_exact(oracle_runs, case):
+    p, Q, K, V, heads = oracle_runs[case]
+    kperm = _stack(heads, "k_perm")
+    Kp = ig.gather(K.cuda(), kperm, p)
+    ref = torch.stack([K[0, h][torch.from_numpy(heads[h].k_perm.astype(np.int64))] for h in range(p.H)])[None]
+    assert torch.equal(Kp.cpu(), ref)
+    ig.device_status()
+
+
+# ------------------------------------------------------------ select/sample
+@pytest.mark.parametrize("case", list(CASES))
+def test_select_sample_bit_exact(oracle_runs, case):
+    p, Q, K, V, heads = oracle_runs[case]
+    m = ig.sample_budget(p)
+    eg, cnt, sp, sb = ig.select_sample(_stack(heads, "cq"), _stack(heads, "ck"), _stack(heads, "k_offsets"), p)
+    eg, cnt, sp, sb = np_(eg)[0], np_(cnt)[0], np_(sp)[0], np_(sb)[0]
+    for h, hr in enumerate(heads):
+        assert np.array_equal(cnt[h], hr.counts), f"head {h} counts"
+        assert np.array_equal(eg[h], hr.exact_groups), f"head {h} exact groups"
+        if m:
+            assert np.array_equal(sp[h], hr.sample_pos), f"head {h} sample positions"
+            valid = hr.sample_pos >= 0
+            np.testing.assert_allclose(sb[h][valid], hr.sample_bias[valid], rtol=1e-5, atol=1e-4)
+            assert np.all(sb[h][~valid] == 0)
+    ig.device_status()
+
+
+def test_select_sample_seed_and_layer_change_draws(oracle_runs):
+    p, Q, K, V, heads = oracle_runs["tiny"]
+    args = (_stack(heads, "cq"), _stack(heads, "ck"), _stack(heads, "k_offsets"))
+    a = np_(ig.select_sample(*args, p)[2])
+    p2 = ig.make_params(1, 1, p.N, p.d, p.Cq, p.Ck, exact_frac=p.exact_frac, sample_frac=p.sample_frac,
+                        seed=p.seed + 1, layer=p.layer)
+    b = np_(ig.select_sample(*args, p2)[2])
+    p3 = ig.make_params(1, 1, p.N, p.d, p.Cq, p.Ck, exact_frac=p.exact_frac, sample_frac=p.sample_frac,
+                        seed=p.seed, layer=p.layer + 1)
+    c = np_(ig.select_sample(*args, p3)[2])
+    assert np.array_equal(a, np_(ig.select_sample(*args, p)[2]))   # reproducible
+    assert not np.array_equal(a, b) and not np.array_equal(a, c)
+
+
+# ------------------------------------------------------------------ k-means
+@pytest.mark.parametrize("case", ["tiny", "ragged_d128", "uniform", "cq1_d64"])
+def test_kmeans_one_step_matches_oracle(oracle_mod, oracle_runs, case):
+    p, Q, K, V, heads = oracle_runs[case]
+    for X, C in ((Q, p.Cq), (K, p.Ck)):
+        Xn = [np_(X[0, h].float()) for h in range(p.H)]
+        init = np.stack([oracle_mod.kmeans_init(x, C) for x in Xn])[None]
+        cent, assign, perm, offs = ig.cluster(X.cuda(), C, 1, p, init=cuda(init))
+        ga = np_(assign)[0]
+        for h in range(p.H):
+            oa, _ = oracle_mod.kmeans_assign(Xn[h], init[0, h])
+            agree = np.mean(ga[h] == oa)
+            assert agree >= 0.999, f"{case} C={C} head {h}: {agree}"
+            # the update from the GPU's own assignment is the mean of its clusters
+            ref = oracle_mod.kmeans_update(Xn[h], oa, init[0, h])
+            same = np.flatnonzero(np.bincount(oa, minlength=C) == np.bincount(ga[h], minlength=C))
+            np.testing.assert_allclose(np_(cent)[0, h][same], ref[same], rtol=0, atol=2e-4)
+            # the returned permutation is the stable sort of the returned assignment
+            assert np.array_equal(np_(perm)[0, h], np.argsort(ga[h], kind="stable"))
+    ig.device_status()
+
+
+def test_kmeans_full_run_invariants(oracle_mod, oracle_runs):
+    p, Q, K, V, heads = oracle_runs["tiny"]
+    X = K
+    cent, assign, perm, offs = ig.cluster(X.cuda(), p.Ck, 10, p)
+    x = np_(X[0, 0].float()).astype(np.float64)
+    a = np_(assign)[0, 0]
+    c = np_(cent)[0, 0]
+    for j in range(p.Ck):
+        if np.any(a == j):
+            np.testing.assert_allclose(c[j], x[a == j].mean(0), rtol=0, atol=2e-4)
+    # same quality as the oracle's own 10-iteration run from the same init
+    inertia = ((x - c[a]) ** 2).sum()
+    o_inertia = ((x - heads[0].ck[heads[0].k_assign].astype(np.float64)) ** 2).sum()
+    assert inertia <= 1.05 * o_inertia
+    agree = np.mean(a == heads[0].k_assign)
+    print(f"10-iteration k-means agreement with the oracle: {agree:.4f}")
+    ig.device_status()
+
+
+# ---------------------------------------------------------------- attention
+def _run_attention_from_oracle(p, Q, K, V, heads):
+    kperm = _stack(heads, "k_perm")
+    Kp = ig.gather(K.cuda(), kperm, p)
+    Vp = ig.gather(V.cuda(), kperm, p)
+    m = ig.sample_budget(p)
+    sp = _stack(heads, "sample_pos") if m else torch.empty((1, p.H, p.Cq, 0), dtype=torch.int32, device="cuda")
+    sb = (_stack(heads, "sample_bias", torch.float32) if m
+          else torch.empty((1, p.H, p.Cq, 0), dtype=torch.float32, device="cuda"))
+    return ig.attention(Q.cuda(), Kp, Vp, _stack(heads, "q_perm"), _stack(heads, "q_offsets"),
+                        _stack(heads, "k_offsets"), _stack(heads, "exact_groups"), _stack(heads, "counts"),
+                        sp, sb, p)
+
+
+def _assert_close(got, ref, what):
+    got = got.astype(np.float64)
+    diff = np.abs(got - ref)
+    mean_rel = diff.sum() / np.abs(ref).sum()
+    assert diff.max() <= MAX_ABS, f"{what}: max abs {diff.max():.3e}"
+    assert mean_rel <= MEAN_REL, f"{what}: mean rel {mean_rel:.3e}"
+    return diff.max(), mean_rel
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_attention_matches_oracle(oracle_runs, case):
+    p, Q, K, V, heads = oracle_runs[case]
+    O = np_(_run_attention_from_oracle(p, Q, K, V, heads).float())[0]
+    for h, hr in enumerate(heads):
+        mx, mr = _assert_close(O[h], hr.out, f"{case} head {h}")
+        print(f"{case} head {h}: max abs {mx:.2e}, mean rel {mr:.2e}")
+    ig.device_status()
+
+
+def test_dense_limit_matches_torch_sdpa():
+    """exact share 1: every key exact, the call is dense softmax attention."""
+    Q, K, V = workloads.random_small(21, 1234, 128, n_centres=6, H=3)
+    p = ig.make_params(1, 3, 1234, 128, 5, 17, iters=3, exact_frac=1.0, sample_frac=0.05)
+    O = ig.forward(Q.cuda(), K.cuda(), V.cuda(), p)
+    ref = torch.softmax(p.softmax_scale * Q.double() @ K.double().transpose(-1, -2), -1) @ V.double()
+    _assert_close(np_(O.float()), ref.numpy(), "dense limit")
+    ig.device_status()
+
+
+# ------------------------------------------------------------------ forward
+@pytest.mark.parametrize("case", ["tiny", "ragged_d128", "uniform"])
+def test_forward_equals_staged_pipeline_and_is_deterministic(case):
+    p, Q, K, V = _inputs(case)
+    Qc, Kc, Vc = Q.cuda(), K.cuda(), V.cuda()
+    ws = torch.empty(ig.workspace_size(p), dtype=torch.uint8, device="cuda")
+    O1 = ig.forward(Qc, Kc, Vc, p, workspace=ws)
+    inter = {k: v.clone() for k, v in ig.forward_intermediates(ws, p).items()}
+    O2 = ig.forward(Qc, Kc, Vc, p)
+    assert torch.equal(O1, O2)
+    cq, qa, qp, qo = ig.cluster(Qc, p.Cq, p.kmeans_iters, p)
+    ck, ka, kp, ko = ig.cluster(Kc, p.Ck, p.kmeans_iters, p)
+    for name, t in (("cq", cq), ("q_assign", qa), ("q_perm", qp), ("q_offsets", qo), ("ck", ck),
+                    ("k_assign", ka), ("k_perm", kp), ("k_offsets", ko)):
+        assert torch.equal(inter[name], t), name
+    Kp, Vp = ig.gather(Kc, kp, p), ig.gather(Vc, kp, p)
+    assert torch.equal(inter["kp"], Kp) and torch.equal(inter["vp"], Vp)
+    eg, cnt, sp, sb = ig.select_sample(cq, ck, ko, p)
+    assert torch.equal(inter["exact_groups"], eg) and torch.equal(inter["counts"], cnt)
+    assert torch.equal(inter["sample_pos"], sp) and torch.equal(inter["sample_bias"], sb)
+    O3 = ig.attention(Qc, Kp, Vp, qp, qo, ko, eg, cnt, sp, sb, p)
+    assert torch.equal(O1, O3)
+    ig.device_status()
+
+
+def test_forward_error_vs_dense_tracks_oracle(oracle_runs):
+    """End to end, the GPU call is as close to dense attention as the oracle's
+    own call on the same inputs (k-means trajectories may differ near ties,
+    so this compares the error level, not elementwise)."""
+    p, Q, K, V, heads = oracle_runs["tiny"]
+    O = np_(ig.forward(Q.cuda(), K.cuda(), V.cuda(), p).float())[0, 0].astype(np.float64)
+    dense = (torch.softmax(p.softmax_scale * Q[0, 0].double() @ K[0, 0].double().T, -1) @ V[0, 0].double()).numpy()
+    e_gpu = np.linalg.norm(O - dense) / np.linalg.norm(dense)
+    e_orc = np.linalg.norm(heads[0].out - dense) / np.linalg.norm(dense)
+    print(f"relative L2 error vs dense: gpu {e_gpu:.4f} oracle {e_orc:.4f}")
+    assert 0.5 * e_orc <= e_gpu <= 2.0 * e_orc
+    ig.device_status()
+
+
+# ------------------------------------------------ full-size sampled parity
+@pytest.mark.slow
+def test_full_size_heads_sampled_parity(oracle_mod):
+    """Wan2.1-14B 720p shape (N=75600, d=128, Cq=100, Ck=500, 16%+16%), heads 0
+    and 39 (noise sigma 0.2 and 0.6): one k-means step from the oracle's
+    initial centroids, select/sample bit-exact from the oracle's centroids,
+    and attention on 96 sampled query rows per head against the oracle."""
+    w = workloads.WAN14B_720P
+    heads = [0, w.H - 1]
+    Q, K, V = workloads.make_inputs(w, heads=heads)
+    H = len(heads)
+    p = ig.make_params(1, H, w.N, w.d, w.Cq, w.Ck, iters=1, exact_frac=w.exact_frac, sample_frac=w.sample_frac,
+                       seed=99, layer=0)
+    rng = np.random.default_rng(0)
+    hr = []
+    for h in range(H):
+        f = lambda t: np_(t[0, h].float())
+        hr.append(_oracle_head(oracle_mod, p, Q, K, V, h, rows=[]))
+    # k-means step from the oracle's init (= the default init)
+    for X, C, attr in ((Q, w.Cq, "q_assign"), (K, w.Ck, "k_assign")):
+        cent, assign, _, _ = ig.cluster(X.cuda(), C, 1, p)
+        ga = np_(assign)[0]
+        for h in range(H):
+            agree = np.mean(ga[h] == getattr(hr[h], attr))
+            assert agree >= 0.999, f"C={C} head {h}: {agree}"
+    # select / sample from the oracle's centroids
+    eg, cnt, sp, sb = ig.select_sample(_stack(hr, "cq"), _stack(hr, "ck"), _stack(hr, "k_offsets"), p)
+    for h in range(H):
+        assert np.array_equal(np_(cnt)[0, h], hr[h].counts)
+        assert np.array_equal(np_(eg)[0, h], hr[h].exact_groups)
+        assert np.array_equal(np_(sp)[0, h], hr[h].sample_pos)
+    # attention with the oracle's lists, sampled rows
+    O = np_(_run_attention_from_oracle(p, Q, K, V, hr).float())[0]
+    for h in range(H):
+        rows = np.sort(rng.choice(w.N, 96, replace=False))
+        ref = oracle_mod.attention_rows(np_(Q[0, h].float()), np_(K[0, h].float()), np_(V[0, h].float()),
+                                        p.softmax_scale, hr[h].q_assign, hr[h].k_perm, hr[h].k_offsets,
+                                        hr[h].exact_groups, hr[h].counts, hr[h].sample_pos, hr[h].sample_bias,
+                                        rows)
+        mx, mr = _assert_close(O[h][rows], ref, f"full-size head {heads[h]}")
+        print(f"full-size head {heads[h]}: max abs {mx:.2e}, mean rel {mr:.2e}")
+    ig.device_status()
