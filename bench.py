@@ -274,7 +274,7 @@ def main():
         evs[1].record(stream)
         ck, ka, kp, ko = ig.cluster(K, w.Ck, w.iters, p)
         evs[2].record(stream)
-        Kp, Vp = ig.gather(K, kp, p), ig.gather(V, kp, p)
+        Kp, Vp = ig.gather(K, kp, p), ig.gather(V, kp, p, to_f16=True)
         evs[3].record(stream)
         eg, cnt, sp, sb = ig.select_sample(cq, ck, ko, p)
         evs[4].record(stream)

@@ -73,7 +73,7 @@ def lib():
         "instagen_device_status": (ctypes.c_int, [vp]),
         "instagen_cluster": (ctypes.c_int, [PP, i32, i32, PP, P, PP, PP, PP, PP, PP, sz, vp]),
         "instagen_permutation": (ctypes.c_int, [PP, i32, P, PP, PP, vp]),
-        "instagen_gather": (ctypes.c_int, [PP, PP, P, PP, vp]),
+        "instagen_gather": (ctypes.c_int, [PP, PP, P, PP, i32, vp]),
         "instagen_select_sample": (ctypes.c_int, [PP, PP, PP, P, PP, PP, PP, PP, vp]),
         "instagen_attention": (ctypes.c_int, [PP, PP, PP, PP, PP, PP, PP, PP, PP, PP, P, PP, vp]),
         "instagen_forward": (ctypes.c_int, [PP, PP, PP, PP, P, PP, sz, vp]),
@@ -187,11 +187,14 @@ def permutation(assign: torch.Tensor, C: int, p: Params):
     return perm, offs
 
 
-def gather(X: torch.Tensor, perm: torch.Tensor, p: Params) -> torch.Tensor:
+def gather(X: torch.Tensor, perm: torch.Tensor, p: Params, to_f16: bool = False) -> torch.Tensor:
+    """Rows of X [B,H,N,d] bf16 in permuted order; fp16 output when to_f16
+    (the layout instagen_attention expects for V)."""
     _need(X, "X", torch.bfloat16, _bhnd(p))
     _need(perm, "perm", torch.int32, (p.B, p.H, p.N))
-    Xp = torch.empty_like(X)
-    _check(lib().instagen_gather(_ptr(X), _ptr(perm), ctypes.byref(p), _ptr(Xp), _stream()), "instagen_gather")
+    Xp = torch.empty(X.shape, dtype=torch.float16 if to_f16 else torch.bfloat16, device=X.device)
+    _check(lib().instagen_gather(_ptr(X), _ptr(perm), ctypes.byref(p), _ptr(Xp), 1 if to_f16 else 0, _stream()),
+           "instagen_gather")
     return Xp
 
 
@@ -215,9 +218,11 @@ def select_sample(cq: torch.Tensor, ck: torch.Tensor, k_offsets: torch.Tensor, p
 
 def attention(Q, Kp, Vp, q_perm, q_offsets, k_offsets, exact_groups, counts, sample_pos, sample_bias,
               p: Params, out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Q original order; Kp, Vp key-cluster order; returns O [B,H,N,d] bf16 (original order)."""
-    for t, n in ((Q, "Q"), (Kp, "Kp"), (Vp, "Vp")):
-        _need(t, n, torch.bfloat16, _bhnd(p))
+    """Q bf16 original order; Kp bf16 and Vp fp16 in key-cluster order (``gather``);
+    returns O [B,H,N,d] bf16 (original order)."""
+    _need(Q, "Q", torch.bfloat16, _bhnd(p))
+    _need(Kp, "Kp", torch.bfloat16, _bhnd(p))
+    _need(Vp, "Vp", torch.float16, _bhnd(p))
     m = sample_budget(p)
     _need(q_perm, "q_perm", torch.int32, (p.B, p.H, p.N))
     _need(q_offsets, "q_offsets", torch.int32, (p.B, p.H, p.Cq + 1))
@@ -271,7 +276,7 @@ def forward_intermediates(workspace: torch.Tensor, p: Params) -> dict:
         q_offsets=view(L.q_offsets, B * H * (Cq + 1), torch.int32, (B, H, Cq + 1)),
         k_offsets=view(L.k_offsets, B * H * (Ck + 1), torch.int32, (B, H, Ck + 1)),
         kp=view(L.kp, B * H * N * d, torch.bfloat16, (B, H, N, d)),
-        vp=view(L.vp, B * H * N * d, torch.bfloat16, (B, H, N, d)),
+        vp=view(L.vp, B * H * N * d, torch.float16, (B, H, N, d)),
         exact_groups=view(L.exact_groups, B * H * Cq * Ck, torch.int32, (B, H, Cq, Ck)),
         counts=view(L.counts, B * H * Cq * 3, torch.int32, (B, H, Cq, 3)),
         sample_pos=view(L.sample_pos, B * H * Cq * m, torch.int32, (B, H, Cq, m)),

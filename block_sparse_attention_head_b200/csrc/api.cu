@@ -7,6 +7,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -223,12 +224,14 @@ int instagen_permutation(const int32_t* assign, int32_t C, const instagen_params
       ig::launch_count_sort(assign, p->B * p->H, p->N, C, perm, offsets, static_cast<cudaStream_t>(stream)));
 }
 
-int instagen_gather(const void* X, const int32_t* perm, const instagen_params* p, void* Xp, void* stream) {
+int instagen_gather(const void* X, const int32_t* perm, const instagen_params* p, void* Xp, int32_t to_f16,
+                    void* stream) {
   int rc = check_params(p);
   if (rc) return rc;
   if (!X || !perm || !Xp || X == Xp || !aligned16(X) || !aligned16(Xp)) return IG_ERR_INVALID_ARG;
+  if (to_f16 != 0 && to_f16 != 1) return IG_ERR_INVALID_ARG;
   return cuda_status(ig::launch_gather_rows(static_cast<const __nv_bfloat16*>(X), nullptr, perm, p->B * p->H,
-                                            p->N, p->d, static_cast<__nv_bfloat16*>(Xp), nullptr,
+                                            p->N, p->d, Xp, nullptr, to_f16 != 0, false,
                                             static_cast<cudaStream_t>(stream)));
 }
 
@@ -280,7 +283,7 @@ int instagen_attention(const void* Q, const void* Kp, const void* Vp, const int3
   ig::AttnArgs a;
   a.Q = static_cast<const __nv_bfloat16*>(Q);
   a.Kp = static_cast<const __nv_bfloat16*>(Kp);
-  a.Vp = static_cast<const __nv_bfloat16*>(Vp);
+  a.Vp = static_cast<const __half*>(Vp);
   a.q_perm = q_perm;
   a.q_offsets = q_offsets;
   a.k_offsets = k_offsets;
@@ -332,8 +335,7 @@ int instagen_forward(const void* Q, const void* K, const void* V, void* O, const
   rc = run_cluster(K, p->Ck, p->kmeans_iters, nullptr, p, ck, ka, kp, ko, cws, cws_bytes, s);
   if (rc) return rc;
   rc = cuda_status(ig::launch_gather_rows(static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V),
-                                          kp, p->B * p->H, p->N, p->d, static_cast<__nv_bfloat16*>(Kp),
-                                          static_cast<__nv_bfloat16*>(Vp), s));
+                                          kp, p->B * p->H, p->N, p->d, Kp, Vp, false, true, s));
   if (rc) return rc;
   rc = instagen_select_sample(cq, ck, ko, p, eg, cnt, sp, sb, stream);
   if (rc) return rc;

@@ -2,6 +2,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -30,9 +31,10 @@ cudaError_t launch_kmeans_update(const KmeansGeom& g, const __nv_bfloat16* X, co
 // ------------------------------------------------------- permutation/gather
 cudaError_t launch_count_sort(const int32_t* assign, int BH, int N, int C, int32_t* perm, int32_t* offsets,
                               cudaStream_t s);
-// Up to two tensors gathered with the same permutation (X1 may be null).
+// Up to two tensors gathered with the same permutation (X1 may be null); a
+// tensor with its f16 flag set is converted bf16 -> fp16.
 cudaError_t launch_gather_rows(const __nv_bfloat16* X0, const __nv_bfloat16* X1, const int32_t* perm, int BH,
-                               int N, int d, __nv_bfloat16* Y0, __nv_bfloat16* Y1, cudaStream_t s);
+                               int N, int d, void* Y0, void* Y1, bool f16_0, bool f16_1, cudaStream_t s);
 
 // ---------------------------------------------------------- select/sample
 struct SelectArgs {
@@ -56,7 +58,7 @@ cudaError_t launch_select_sample(const SelectArgs& a, cudaStream_t s);
 struct AttnArgs {
   const __nv_bfloat16* Q;
   const __nv_bfloat16* Kp;
-  const __nv_bfloat16* Vp;
+  const __half* Vp;  // fp16 (converted by the gather)
   const int32_t* q_perm;
   const int32_t* q_offsets;
   const int32_t* k_offsets;

@@ -95,10 +95,29 @@ cudaError_t launch_count_sort(const int32_t* assign, int BH, int N, int C, int32
 
 // ---------------------------------------------------------------- gather
 // Y[bh, p, :] = X[bh, perm[bh, p], :] for one or two tensors; each thread moves
-// 16 bytes, consecutive threads move consecutive chunks of a row.
+// 16 bytes, consecutive threads move consecutive chunks of a row.  A tensor
+// whose `to_f16` flag is set is converted from bf16 to fp16 on the way
+// (values beyond the fp16 range are saturated and reported).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+  uint4 out;
+  uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+  bool over = false;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    float2 f = __bfloat1622float2(h[e]);
+    over |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
+    f.x = fminf(fmaxf(f.x, -65504.f), 65504.f);
+    f.y = fminf(fmaxf(f.y, -65504.f), 65504.f);
+    o[e] = pack_f16x2(f.x, f.y);
+  }
+  if (over) raise_error(kErrRange);
+  return out;
+}
+
 __global__ void gather_rows_kernel(const uint4* __restrict__ X0, const uint4* __restrict__ X1,
                                    const int32_t* __restrict__ perm, long long rows, int N, int cpr,
-                                   uint4* __restrict__ Y0, uint4* __restrict__ Y1) {
+                                   uint4* __restrict__ Y0, uint4* __restrict__ Y1, int f16_0, int f16_1) {
   const long long total = rows * cpr;
   for (long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x; g < total;
        g += (long long)gridDim.x * blockDim.x) {
@@ -111,13 +130,17 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ X0, const uint4* __
       continue;
     }
     const long long si = (bh * N + src) * cpr + ch;
-    Y0[g] = X0[si];
-    if (X1) Y1[g] = X1[si];
+    const uint4 v0 = X0[si];
+    Y0[g] = f16_0 ? bf16x8_to_f16x8(v0) : v0;
+    if (X1) {
+      const uint4 v1 = X1[si];
+      Y1[g] = f16_1 ? bf16x8_to_f16x8(v1) : v1;
+    }
   }
 }
 
 cudaError_t launch_gather_rows(const __nv_bfloat16* X0, const __nv_bfloat16* X1, const int32_t* perm, int BH,
-                               int N, int d, __nv_bfloat16* Y0, __nv_bfloat16* Y1, cudaStream_t s) {
+                               int N, int d, void* Y0, void* Y1, bool f16_0, bool f16_1, cudaStream_t s) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -131,7 +154,7 @@ cudaError_t launch_gather_rows(const __nv_bfloat16* X0, const __nv_bfloat16* X1,
   if (blocks < 1) blocks = 1;
   gather_rows_kernel<<<(unsigned)blocks, threads, 0, s>>>(
       reinterpret_cast<const uint4*>(X0), reinterpret_cast<const uint4*>(X1), perm, rows, N, cpr,
-      reinterpret_cast<uint4*>(Y0), reinterpret_cast<uint4*>(Y1));
+      reinterpret_cast<uint4*>(Y0), reinterpret_cast<uint4*>(Y1), f16_0 ? 1 : 0, f16_1 ? 1 : 0);
   return cudaGetLastError();
 }
 

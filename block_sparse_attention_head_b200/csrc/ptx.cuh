@@ -6,6 +6,7 @@
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace ig {
 
@@ -13,11 +14,12 @@ constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
 
 // Device error word shared by every kernel of the library (read and cleared by
 // instagen_device_status).  Codes: bit 0 wait timeout, bit 1 index out of range,
-// bit 2 invalid sampling state.
+// bit 2 invalid sampling state, bit 3 value outside the fp16 range.
 __device__ int g_device_error = 0;
 constexpr int kErrTimeout = 1;
 constexpr int kErrIndex = 2;
 constexpr int kErrSampling = 4;
+constexpr int kErrRange = 8;
 
 __device__ __forceinline__ void raise_error(int code) { atomicOr(&g_device_error, code); }
 
@@ -203,11 +205,13 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
+// Instruction descriptor, kind::f16: fp32 accumulator, A and B both bf16
+// (f16_operands = false) or both fp16 (true).
+__host__ __device__ constexpr uint32_t umma_idesc_f16kind(int M, int N, bool a_mn_major, bool b_mn_major,
+                                                          bool f16_operands) {
   return (1u << 4)                                  // D format: f32
-         | (1u << 7)                                // A: bf16
-         | (1u << 10)                               // B: bf16
+         | ((f16_operands ? 0u : 1u) << 7)          // A: 0 = f16, 1 = bf16
+         | ((f16_operands ? 0u : 1u) << 10)         // B: 0 = f16, 1 = bf16
          | ((a_mn_major ? 1u : 0u) << 15)           // A major
          | ((b_mn_major ? 1u : 0u) << 16)           // B major
          | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
@@ -225,6 +229,15 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return umma_idesc_f16kind(M, N, a_mn_major, b_mn_major, false);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);  // .x = lo (low 16 bits)
+  return *reinterpret_cast<uint32_t*>(&v);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

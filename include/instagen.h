@@ -120,9 +120,13 @@ int instagen_permutation(const int32_t* assign, int32_t C, const instagen_params
 
 /*
  * Gather rows into permuted order: Xp[bh, s, :] = X[bh, perm[bh, s], :].
- *   X, Xp [B,H,N,d] bf16 (distinct buffers); perm [B,H,N] int32.
+ *   X [B,H,N,d] bf16; perm [B,H,N] int32; Xp [B,H,N,d] (distinct buffer):
+ *   bf16 when to_f16 = 0 (keys), fp16 when to_f16 = 1 (values: the attention
+ *   kernel multiplies fp16 P by fp16 V).  Values beyond the fp16 range are
+ *   saturated to +-65504 and reported as IG_ERR_DEVICE_CHECK.
  */
-int instagen_gather(const void* X, const int32_t* perm, const instagen_params* p, void* Xp, void* stream);
+int instagen_gather(const void* X, const int32_t* perm, const instagen_params* p, void* Xp, int32_t to_f16,
+                    void* stream);
 
 /*
  * (b)+(c) Centroid scores, exact set and the group-shared sample
@@ -159,15 +163,17 @@ int instagen_select_sample(const float* cq, const float* ck, const int32_t* k_of
  *   online-softmax pass (Figure 3 (d); "computes them together with the top-k
  *   blocks in a single attention kernel", ICLR listing abstract).
  *   Q  [B,H,N,d] bf16 in ORIGINAL token order (rows gathered via q_perm).
- *   Kp, Vp [B,H,N,d] bf16 in key-cluster (permuted) order (instagen_gather).
+ *   Kp [B,H,N,d] bf16 and Vp [B,H,N,d] fp16, both in key-cluster (permuted)
+ *   order (instagen_gather with to_f16 = 0 and 1).
  *   q_perm, q_offsets: query permutation; k_offsets: key cluster ranges.
  *   exact_groups, counts, sample_pos, sample_bias: as instagen_select_sample.
  *   O  [B,H,N,d] bf16 out, ORIGINAL token order.  Query q of group i gets
  *   softmax over {scale*q.k : k in exact groups of i} U {scale*q.k_t + bias_t :
  *   sample slots t of i} applied to the matching V rows (a key drawn twice
  *   counts twice).
- * QK^T and PV run on the tcgen05 tensor cores (bf16 in, fp32 accumulate in
- * TMEM); P is rounded to bf16 for the PV product.
+ * QK^T runs on the tcgen05 tensor cores with bf16 operands and PV with fp16
+ * operands (P = exp2 of the shifted logits, <= 256, rounded to fp16), both
+ * accumulating in fp32 in TMEM; O is rounded to bf16 once at the end.
  */
 int instagen_attention(const void* Q, const void* Kp, const void* Vp, const int32_t* q_perm,
                        const int32_t* q_offsets, const int32_t* k_offsets, const int32_t* exact_groups,
@@ -190,7 +196,7 @@ typedef struct {
   size_t q_assign, k_assign;     /* int32 [B,H,N]                               */
   size_t q_perm, k_perm;         /* int32 [B,H,N]                               */
   size_t q_offsets, k_offsets;   /* int32 [B,H,Cq+1], [B,H,Ck+1]                */
-  size_t kp, vp;                 /* bf16 [B,H,N,d] permuted K and V             */
+  size_t kp, vp;                 /* [B,H,N,d] permuted K (bf16) and V (fp16)    */
   size_t exact_groups, counts;   /* int32 [B,H,Cq,Ck], [B,H,Cq,3]               */
   size_t sample_pos, sample_bias;/* int32 / fp32 [B,H,Cq,m]                     */
   size_t cluster_ws;             /* scratch for instagen_cluster                */

@@ -80,7 +80,8 @@ def test_null_pointers_and_workspace_rejected(lib):
     assert lib.instagen_forward(fake, fake, fake, fake, ctypes.byref(p), fake, 16, None) == 3
     assert lib.instagen_cluster(None, 8, 1, None, ctypes.byref(p), None, None, None, None, None, 0, None) == 1
     assert lib.instagen_cluster(fake, 8, 0, None, ctypes.byref(p), fake, fake, fake, fake, fake, 0, None) == 1
-    assert lib.instagen_gather(fake, fake, ctypes.byref(p), fake, None) == 1      # X == Xp
+    assert lib.instagen_gather(fake, fake, ctypes.byref(p), fake, 0, None) == 1   # X == Xp
+    assert lib.instagen_gather(fake, fake, ctypes.byref(p), ctypes.c_void_p(1 << 21), 2, None) == 1  # bad flag
     assert lib.instagen_select_sample(None, None, None, ctypes.byref(p), None, None, None, None, None) == 1
     big = ig.make_params(1, 2, 1000, 64, 8, 3000)
     assert lib.instagen_attention(fake, fake, fake, fake, fake, fake, fake, fake, fake, fake,

@@ -121,7 +121,23 @@ def test_gather_exact(oracle_runs, case):
     Kp = ig.gather(K.cuda(), kperm, p)
     ref = torch.stack([K[0, h][torch.from_numpy(heads[h].k_perm.astype(np.int64))] for h in range(p.H)])[None]
     assert torch.equal(Kp.cpu(), ref)
+    Vp = ig.gather(V.cuda(), kperm, p, to_f16=True)
+    refv = torch.stack([V[0, h][torch.from_numpy(heads[h].k_perm.astype(np.int64))] for h in range(p.H)])[None]
+    assert Vp.dtype == torch.float16 and torch.equal(Vp.cpu(), refv.to(torch.float16))
     ig.device_status()
+
+
+def test_gather_f16_saturates_and_reports():
+    p = ig.make_params(1, 1, 64, 64, 2, 2)
+    X = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16)
+    X[0, 0, 5, 3] = 1e6
+    X[0, 0, 9, 1] = -3e5
+    perm = torch.arange(64, dtype=torch.int32)[None, None].cuda()
+    Y = ig.gather(X.cuda(), perm, p, to_f16=True).cpu()
+    assert Y[0, 0, 5, 3].item() == 65504.0 and Y[0, 0, 9, 1].item() == -65504.0
+    with pytest.raises(ig.InstaGenError, match="device check"):
+        ig.device_status()
+    ig.device_status()  # the error word was cleared
 
 
 # ------------------------------------------------------------ select/sample
@@ -201,7 +217,7 @@ def test_kmeans_full_run_invariants(oracle_mod, oracle_runs):
 def _run_attention_from_oracle(p, Q, K, V, heads):
     kperm = _stack(heads, "k_perm")
     Kp = ig.gather(K.cuda(), kperm, p)
-    Vp = ig.gather(V.cuda(), kperm, p)
+    Vp = ig.gather(V.cuda(), kperm, p, to_f16=True)
     m = ig.sample_budget(p)
     sp = _stack(heads, "sample_pos") if m else torch.empty((1, p.H, p.Cq, 0), dtype=torch.int32, device="cuda")
     sb = (_stack(heads, "sample_bias", torch.float32) if m
@@ -255,7 +271,7 @@ def test_forward_equals_staged_pipeline_and_is_deterministic(case):
     for name, t in (("cq", cq), ("q_assign", qa), ("q_perm", qp), ("q_offsets", qo), ("ck", ck),
                     ("k_assign", ka), ("k_perm", kp), ("k_offsets", ko)):
         assert torch.equal(inter[name], t), name
-    Kp, Vp = ig.gather(Kc, kp, p), ig.gather(Vc, kp, p)
+    Kp, Vp = ig.gather(Kc, kp, p), ig.gather(Vc, kp, p, to_f16=True)
     assert torch.equal(inter["kp"], Kp) and torch.equal(inter["vp"], Vp)
     eg, cnt, sp, sb = ig.select_sample(cq, ck, ko, p)
     assert torch.equal(inter["exact_groups"], eg) and torch.equal(inter["counts"], cnt)
