@@ -5,48 +5,53 @@
 // "computed together with the top-k blocks in a single attention kernel, with
 // sampled scores reweighted to account for the full skipped region").
 //
-// CTA = one tile of 128 queries of one query group (rows gathered from Q via
-// the query permutation).  The group's key list is its exact groups (in rank
-// order, contiguous ranges of the permuted K/V) followed by its m sample slots
-// (gathered rows, with log-weight); it is walked in tiles of 128 keys:
-//   S = Q K^T          tcgen05 (M=128, N=128, K=d), fp32 in TMEM (2 buffers)
-//   P = 2^(S*scale*log2e + bias*log2e - m_run)   softmax warps, fp16 -> smem
-//   O += P V           tcgen05 (M=128, N=d, K=128), fp16 operands, fp32 in TMEM
-// P and V are fp16 (V converted by the gather): P <= 256 keeps 11 mantissa
-// bits instead of bf16's 8, which keeps the output within 2e-3 mean relative
-// error of exact arithmetic once it is rounded to bf16.
-// The running max is only raised when it grows by more than 8 (log2 units), so
-// P <= 256 and the O rescale (a TMEM read-modify-write) is rare.
+// CTA = two tiles of 128 queries (Q0, Q1) of one query group, gathered from Q
+// through the query permutation.  Both share the group's key list: its exact
+// groups (rank order; contiguous ranges of the permuted K/V) followed by its m
+// sample slots (gathered rows with log-weight), walked in tiles of 128 keys.
+// Per key tile j and query tile t:
+//   S_t = Q_t K_j^T        tcgen05 (M=128, N=128, K=d, bf16), fp32 in TMEM
+//   P_t = 2^(S_t*scale*log2e + bias*log2e - m_t)    softmax warpgroup t,
+//                          written back as fp16 into S_t's TMEM columns
+//   O_t += P_t V_j         tcgen05 with A (P_t) read from TMEM, fp16 operands
+// The tensor pipe alternates [PV_0(j-1), S_0(j)] and [PV_1(j-1), S_1(j)], so
+// one warpgroup's softmax runs while the other tile's MMAs execute.  The
+// running max is only raised when it grows by more than 8 (log2 units), so
+// P <= 256 and the O rescale (a TMEM read-modify-write) is rare; it is done by
+// the softmax warpgroup after S_t(j) lands, which the MMA pipe orders after
+// PV_t(j-1).  P and V are fp16 (V converted by the gather): 11 mantissa bits
+// keep the output within 2e-3 mean relative error after its bf16 rounding.
 //
-// Warps: 0-1 producer (cp.async 16-byte row gathers, 128-byte swizzle; two
-// rows per thread), 2 MMA issuer + TMEM owner, 3 idle, 4-7 softmax (thread =
-// query row = TMEM lane).  Eight warps leave every thread 255 registers.
+// Warps: 0 MMA issuer + TMEM owner, 1 idle, 2-3 producer (cp.async 16-byte
+// row gathers into the 128-byte-swizzled operand layout, completion tracked
+// by the stage mbarriers so the producer never blocks on memory), 4-7
+// softmax for Q0, 8-11 softmax for Q1 (thread = query row = TMEM lane).
 #include "internal.cuh"
 #include "ptx.cuh"
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace ig {
 
 namespace {
-constexpr int kAttnThreads = 256;
+constexpr int kAttnThreads = 384;
 constexpr int kProducers = 64;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;
 
 template <int D>
 struct AttnSmem {
-  static constexpr int kTileBytes = D * 256;  // 128 rows x D bf16
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileBytes;          // 2 stages
-  static constexpr int kV = kK + 2 * kTileBytes;      // 2 stages
-  static constexpr int kP = kV + 2 * kTileBytes;      // 128 x 128 bf16
-  static constexpr int kBias = kP + 32768;            // 4 warps x 2 buffers x 128 fp32
-  static constexpr int kGStart = kBias + 4096;        // exact group start slots
-  static constexpr int kGPre = kGStart + kAttnMaxExactGroups * 4;  // exclusive prefix of sizes
-  static constexpr int kBars = kGPre + (kAttnMaxExactGroups + 1) * 4 + 12;  // 8-B aligned below
+  static constexpr int kTileBytes = D * 256;  // 128 rows x D 16-bit
+  static constexpr int kQ = 0;                          // 2 query tiles
+  static constexpr int kK = kQ + 2 * kTileBytes;        // 2 stages
+  static constexpr int kV = kK + 2 * kTileBytes;        // 2 stages
+  static constexpr int kGStart = kV + 2 * kTileBytes;   // exact group start slots
+  static constexpr int kGPre = kGStart + kAttnMaxExactGroups * 4;         // exclusive prefix of sizes
+  static constexpr int kBias = kGPre + (kAttnMaxExactGroups + 1) * 4 + 12;  // 8 warps x 2 x 128 fp32
+  static constexpr int kBars = kBias + 8 * 2 * 128 * 4;
   static constexpr int kNumBars = 16;
-  static constexpr int kMisc = ((kBars + 7) & ~7) + kNumBars * 8;
+  static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kBytes = kMisc + 64;
   static size_t bytes() { return 1024 + kBytes; }
 };
@@ -60,45 +65,45 @@ __device__ __forceinline__ const T* row_ptr(const T* base, int bh, int N, int ro
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) {
   using L = AttnSmem<D>;
+  static_assert(L::kBars % 8 == 0, "barrier alignment");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* bias_s = reinterpret_cast<float*>(smem + L::kBias);
   int* gstart = reinterpret_cast<int*>(smem + L::kGStart);
   int* gpre = reinterpret_cast<int*>(smem + L::kGPre);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ((L::kBars + 7) & ~7));
+  float* bias_s = reinterpret_cast<float*>(smem + L::kBias);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;   // [2]
+  uint64_t* k_full = bars + 1;   // [2] stages
   uint64_t* k_empty = bars + 3;  // [2]
   uint64_t* v_full = bars + 5;   // [2]
   uint64_t* v_empty = bars + 7;  // [2]
-  uint64_t* s_full = bars + 9;   // [2]
-  uint64_t* s_free = bars + 11;  // [2]
-  uint64_t* p_full = bars + 13;
-  uint64_t* pv_done = bars + 14;
-  uint64_t* fin = bars + 15;
+  uint64_t* s_full = bars + 9;   // [2] query tiles
+  uint64_t* p_full = bars + 11;  // [2] query tiles
+  uint64_t* o_done = bars + 13;
+  uint64_t* fin = bars + 14;
   int* misc = reinterpret_cast<int*>(smem + L::kMisc);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc + 0);
   volatile int* abort_flag = misc + 1;
-  int* work = misc + 2;  // group, local tile
+  int* work = misc + 2;  // group, local pair
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.y, t_glob = blockIdx.x;
   const int N = a.N, Cq = a.Cq, Ck = a.Ck;
 
-  // ---- which (query group, tile) this CTA owns: prefix of ceil(n_i/128)
+  // ---- which (query group, pair of query tiles) this CTA owns
   if (warp == 0) {
     const int32_t* qoff = a.q_offsets + (size_t)bh * (Cq + 1);
     int run = 0, found_g = -1, found_t = 0;
     for (int c0 = 0; c0 < Cq && found_g < 0; c0 += 32) {
       const int c = c0 + lane;
-      const int nt = (c < Cq) ? (qoff[c + 1] - qoff[c] + 127) / 128 : 0;
-      int incl = nt;
+      const int np = (c < Cq) ? (qoff[c + 1] - qoff[c] + 255) / 256 : 0;
+      int incl = np;
       for (int o = 1; o < 32; o <<= 1) {
         const int v = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += v;
       }
-      const int excl = run + incl - nt;
-      const bool mine = nt > 0 && t_glob >= excl && t_glob < excl + nt;
+      const int excl = run + incl - np;
+      const bool mine = np > 0 && t_glob >= excl && t_glob < excl + np;
       const unsigned hit = __ballot_sync(0xffffffffu, mine);
       if (hit) {
         const int src = __ffs(hit) - 1;
@@ -114,16 +119,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
   }
   __syncthreads();
   const int gi = work[0];
-  if (gi < 0) return;  // tile index beyond this head's tiles
-  const int lt = work[1];
+  if (gi < 0) return;  // pair index beyond this head's pairs
+  const int lp = work[1];
   const size_t grp = (size_t)bh * Cq + gi;
   const int qlo = a.q_offsets[(size_t)bh * (Cq + 1) + gi];
   const int qhi = a.q_offsets[(size_t)bh * (Cq + 1) + gi + 1];
-  const int q0 = qlo + lt * 128;
-  const int nrows = min(128, qhi - q0);
+  const int q0 = qlo + lp * 256;
+  const int rows0 = min(128, qhi - q0);
+  const int rows1 = max(0, min(128, qhi - q0 - 128));
+  const int ntiles = rows1 > 0 ? 2 : 1;
   const int n_exact = a.counts[grp * 3 + 0];
   const int ns = a.counts[grp * 3 + 2];
-  if (qlo < 0 || qhi > N || nrows < 1 || n_exact < 1 || n_exact > Ck || n_exact > kAttnMaxExactGroups || ns < 0 ||
+  if (qlo < 0 || qhi > N || rows0 < 1 || n_exact < 1 || n_exact > Ck || n_exact > kAttnMaxExactGroups || ns < 0 ||
       ns > a.m) {
     if (tid == 0) raise_error(kErrIndex);
     return;
@@ -159,7 +166,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
     }
     if (lane == 0) gpre[n_exact] = run;
   }
-  if (tid == 0) {
+  if (tid == 32) {
     mbar_init(q_full, kProducers);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], kProducers);
@@ -167,15 +174,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
       mbar_init(&k_empty[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 128);
+      mbar_init(&p_full[s], 128);
     }
-    mbar_init(p_full, 128);
-    mbar_init(pv_done, 1);
+    mbar_init(o_done, 1);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 2) {
+  if (warp == 0) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
@@ -183,24 +189,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const int Xi = gpre[n_exact];             // exact keys
-  const int Lk = Xi + ns;                    // keys in the list
-  const int ntk = (Lk + 127) / 128;          // key tiles (>= 1)
+  const int Xi = gpre[n_exact];     // exact keys
+  const int Lk = Xi + ns;           // keys in the list
+  const int ntk = (Lk + 127) / 128; // key tiles
   const uint32_t q_s = smem_u32(smem + L::kQ);
   const uint32_t k_s = smem_u32(smem + L::kK);
   const uint32_t v_s = smem_u32(smem + L::kV);
-  const uint32_t p_s = smem_u32(smem + L::kP);
   const int32_t* spos = a.sample_pos + grp * (size_t)a.m;
   const float* sbias = a.sample_bias + grp * (size_t)a.m;
 
   if (ntk < 1) {
     if (tid == 0) raise_error(kErrIndex);  // empty key list: nothing to attend
-  } else if (warp < 2) {
+  } else if (warp == 2 || warp == 3) {
     // ================================================================ producer
-    // thread t handles tile rows t and t + 64
-    for (int h = 0; h < 2; ++h) {
-      const int r = tid + h * kProducers;
-      bool valid = r < nrows;
+    const int tp = tid - 64;  // 0..63: rows tp and tp + 64 of every K/V tile
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {  // query rows tp + 64h of the 256-row pair
+      const int r = tp + 64 * h;
+      const int t = r >> 7, rr = r & 127;
+      bool valid = rr < (t == 0 ? rows0 : rows1);
       int tok = 0;
       if (valid) {
         tok = a.q_perm[(size_t)bh * N + q0 + r];
@@ -211,19 +218,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
         }
       }
       const __nv_bfloat16* src = row_ptr(a.Q, bh, N, tok, D);
+      const uint32_t dst = q_s + t * L::kTileBytes;
 #pragma unroll
       for (int c = 0; c < D / 8; ++c)
-        cp_async_16(q_s + (c >> 3) * 16384 + sw128_offset(r, c & 7), src + c * 8, valid ? 16u : 0u);
+        cp_async_16(dst + (c >> 3) * 16384 + sw128_offset(rr, c & 7), src + c * 8, valid ? 16u : 0u);
     }
-    cp_async_commit();
-    bool ok = true;
-    for (int kt = 0; kt < ntk && ok; ++kt) {
+    cp_async_arrive_noinc(q_full);
+    for (int kt = 0; kt < ntk; ++kt) {
       const int s = kt & 1, use = kt >> 1;
       int pos[2];
       bool valid[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int l = kt * 128 + tid + h * kProducers;  // key slot of this row in the list
+        const int l = kt * 128 + tp + h * kProducers;  // slot of this row in the key list
         int p = -1;
         if (l < Xi) {
           int lo = 0, hi = n_exact - 1;  // last e with gpre[e] <= l
@@ -246,58 +253,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
         pos[h] = v ? p : 0;
         valid[h] = v;
       }
-      if (kt >= 2 && !mbar_wait(&k_empty[s], (use - 1) & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
+      if (kt >= 2 && !mbar_wait(&k_empty[s], (use - 1) & 1, abort_flag)) break;
       const uint32_t kdst = k_s + s * L::kTileBytes;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int r = tid + h * kProducers;
+        const int r = tp + h * kProducers;
         const __nv_bfloat16* ksrc = row_ptr(a.Kp, bh, N, pos[h], D);
 #pragma unroll
         for (int c = 0; c < D / 8; ++c)
           cp_async_16(kdst + (c >> 3) * 16384 + sw128_offset(r, c & 7), ksrc + c * 8, valid[h] ? 16u : 0u);
       }
-      cp_async_commit();
-      cp_async_wait<1>();  // the previous group (Q or V of the last tile) has landed
-      fence_proxy_async_smem();
-      mbar_arrive(kt == 0 ? q_full : &v_full[(kt - 1) & 1]);
-      if (kt >= 2 && !mbar_wait(&v_empty[s], (use - 1) & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
+      cp_async_arrive_noinc(&k_full[s]);
+      if (kt >= 2 && !mbar_wait(&v_empty[s], (use - 1) & 1, abort_flag)) break;
       const uint32_t vdst = v_s + s * L::kTileBytes;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int r = tid + h * kProducers;
+        const int r = tp + h * kProducers;
         const __half* vsrc = row_ptr(a.Vp, bh, N, pos[h], D);
 #pragma unroll
         for (int c = 0; c < D / 8; ++c)
           cp_async_16(vdst + (c >> 3) * 16384 + sw128_offset(r, c & 7), vsrc + c * 8, valid[h] ? 16u : 0u);
       }
-      cp_async_commit();
-      cp_async_wait<1>();  // this tile's K has landed
-      fence_proxy_async_smem();
-      mbar_arrive(&k_full[s]);
+      cp_async_arrive_noinc(&v_full[s]);
     }
-    cp_async_wait<0>();
-    if (ok) {
-      fence_proxy_async_smem();
-      mbar_arrive(&v_full[(ntk - 1) & 1]);
-    }
+    cp_async_wait_all();
   } else if (warp >= 4) {
     // ================================================================= softmax
-    const int r = tid - 128;  // query row == TMEM lane
+    const int t = (warp - 4) >> 2;          // query tile of this warpgroup
+    const int r = tid - 128 - 128 * t;      // query row == TMEM lane
     const uint32_t lane_off = (uint32_t)((r & ~31) << 16);
+    const uint32_t s_col = tmem + lane_off + (uint32_t)(128 * t);
+    const uint32_t o_col = tmem + lane_off + (uint32_t)(256 + 128 * t);
+    const bool active = t < ntiles;
     float m_run = -__int_as_float(0x7f800000);
     float l_run = 0.f;
-    bool ok = true;
-    for (int kt = 0; kt < ntk; ++kt) {
-      const int sb = kt & 1;
-      // this warp's private copy of the tile's column log-weights (log2 units);
-      // warp-local so an aborting thread can never strand the others
-      float* wb = bias_s + ((warp - 4) * 2 + sb) * 128;
+    bool ok = active;
+    for (int kt = 0; kt < ntk && ok; ++kt) {
+      // this warp's private copy of the tile's column log-weights (log2 units)
+      float* wb = bias_s + ((warp - 4) * 2 + (kt & 1)) * 128;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int l = kt * 128 + lane * 4 + e;
@@ -311,27 +304,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
         wb[lane * 4 + e] = b;
       }
       __syncwarp();
-      if (!mbar_wait_warp(&s_full[sb], (kt >> 1) & 1, abort_flag)) {
+      if (!mbar_wait_warp(&s_full[t], kt & 1, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float x[128];
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tmem + lane_off + sb * 128 + c4 * 32, x + c4 * 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&s_free[sb]);
-      const float4* bsv = reinterpret_cast<const float4*>(wb);
+      const float4* b4 = reinterpret_cast<const float4*>(wb);
+      // pass 1: row maximum of the scaled, reweighted logits
       float mx = -__int_as_float(0x7f800000);
+#pragma unroll 1
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float v[32];
+        tmem_ld32(s_col + c4 * 32, v);
+        tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 128; c += 4) {
-        const float4 b4 = bsv[c >> 2];
-        x[c + 0] = fmaf(x[c + 0], a.scale_log2, b4.x);
-        x[c + 1] = fmaf(x[c + 1], a.scale_log2, b4.y);
-        x[c + 2] = fmaf(x[c + 2], a.scale_log2, b4.z);
-        x[c + 3] = fmaf(x[c + 3], a.scale_log2, b4.w);
-        mx = fmaxf(mx, fmaxf(fmaxf(x[c], x[c + 1]), fmaxf(x[c + 2], x[c + 3])));
+        for (int e = 0; e < 32; e += 4) {
+          const float4 bb = b4[(c4 * 32 + e) >> 2];
+          mx = fmaxf(mx, fmaxf(fmaxf(fmaf(v[e], a.scale_log2, bb.x), fmaf(v[e + 1], a.scale_log2, bb.y)),
+                               fmaxf(fmaf(v[e + 2], a.scale_log2, bb.z), fmaf(v[e + 3], a.scale_log2, bb.w))));
+        }
       }
       const float m_new = fmaxf(m_run, mx);
       const bool rescale = m_new > m_run + kRescaleThreshold;
@@ -340,59 +331,60 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
         alpha = ex2_approx(m_run - m_new);
         m_run = m_new;
       }
+      // O_t holds PV_t(kt-1) (the MMA pipe ran it before S_t(kt)); tcgen05.ld/st
+      // are warp-collective, so the warp rescales if any of its rows needs it
+      if (kt >= 1 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+        for (int c4 = 0; c4 < D / 32; ++c4) {
+          float o[32];
+          tmem_ld32(o_col + c4 * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] *= alpha;
+          tmem_st32(o_col + c4 * 32, o);
+        }
+      }
+      // pass 2: P = 2^(x - m) as fp16 pairs into the first 64 columns of S_t
       float rs = 0.f;
+#pragma unroll 1
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float v[32];
+        tmem_ld32(s_col + c4 * 32, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        x[c] = ex2_approx(x[c] - m_run);
-        rs += x[c];
+        for (int e = 0; e < 32; e += 4) {
+          const float4 bb = b4[(c4 * 32 + e) >> 2];
+          const float p0 = ex2_approx(fmaf(v[e], a.scale_log2, bb.x) - m_run);
+          const float p1 = ex2_approx(fmaf(v[e + 1], a.scale_log2, bb.y) - m_run);
+          const float p2 = ex2_approx(fmaf(v[e + 2], a.scale_log2, bb.z) - m_run);
+          const float p3 = ex2_approx(fmaf(v[e + 3], a.scale_log2, bb.w) - m_run);
+          rs += (p0 + p1) + (p2 + p3);
+          pk[e >> 1] = pack_f16x2(p0, p1);
+          pk[(e >> 1) + 1] = pack_f16x2(p2, p3);
+        }
+        tmem_st16(s_col + c4 * 16, pk);
       }
+      tmem_wait_st();
       l_run = l_run * alpha + rs;
-      if (kt >= 1) {
-        if (!mbar_wait_warp(pv_done, (kt - 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // tcgen05.ld/st are warp-collective: the warp rescales if any of its
-        // rows needs it (alpha is 1 for the others)
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-          for (int c4 = 0; c4 < D / 32; ++c4) {
-            float o[32];
-            const uint32_t oaddr = tmem + lane_off + 256 + c4 * 32;
-            tmem_ld32(oaddr, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(oaddr, o);
-          }
-          tmem_wait_st();
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const uint32_t addr = p_s + (c >> 3) * 16384 + sw128_offset(r, c & 7);
-        st_shared_v4(addr, pack_f16x2(x[8 * c + 0], x[8 * c + 1]), pack_f16x2(x[8 * c + 2], x[8 * c + 3]),
-                     pack_f16x2(x[8 * c + 4], x[8 * c + 5]), pack_f16x2(x[8 * c + 6], x[8 * c + 7]));
-      }
-      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[t]);
     }
-    if (ok && mbar_wait_warp(pv_done, (ntk - 1) & 1, abort_flag)) {
+    if (ok && mbar_wait_warp(o_done, 0, abort_flag)) {
       tc_fence_after();
       const float inv = 1.f / l_run;
+      const int nrows = t == 0 ? rows0 : rows1;
       bool valid = r < nrows;
       int tok = 0;
       if (valid) {
-        tok = a.q_perm[(size_t)bh * N + q0 + r];
+        tok = a.q_perm[(size_t)bh * N + q0 + 128 * t + r];
         if (tok < 0 || tok >= N) valid = false;
       }
       __nv_bfloat16* dst = a.O + ((size_t)bh * N + tok) * D;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
         float o[32];
-        tmem_ld32(tmem + lane_off + 256 + c4 * 32, o);
+        tmem_ld32(o_col + c4 * 32, o);
         tmem_wait_ld();
         if (valid) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c4 * 32);
@@ -406,55 +398,64 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
         }
       }
     }
-  } else if (warp == 2 && lane == 0) {
+  } else if (warp == 0 && lane == 0) {
     // ===================================================================== MMA
     const uint32_t idesc_qk = umma_idesc_bf16(128, 128, false, false);
-    const uint32_t idesc_pv = umma_idesc_f16kind(128, D, false, true, true);  // fp16 P and V
+    const uint32_t idesc_pv = umma_idesc_f16kind(128, D, false, true, true);  // fp16 P (TMEM) x fp16 V
     bool ok = mbar_wait(q_full, 0, abort_flag);
-    auto issue_pv = [&](int j) -> bool {
-      if (!mbar_wait(p_full, j & 1, abort_flag)) return false;
-      if (!mbar_wait(&v_full[j & 1], (j >> 1) & 1, abort_flag)) return false;
+    fence_proxy_async_smem();
+    // O_t += P_t(j) V(j), A operand = P_t in TMEM (columns of S_t)
+    auto issue_pv = [&](int t, int j) -> bool {
+      if (!mbar_wait(&p_full[t], j & 1, abort_flag)) return false;
       tc_fence_after();
       const uint32_t vb = v_s + (j & 1) * L::kTileBytes;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const uint64_t ad = umma_desc_sw128(p_s + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
         const uint64_t bd = umma_desc_sw128(vb + k * 2048, 16384, 1024);
-        umma_bf16_ss(tmem + 256, ad, bd, idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
+        umma_f16_ts(tmem + 256 + 128 * t, tmem + 128 * t + 8 * k, bd, idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
       }
-      umma_commit(&v_empty[j & 1]);
-      umma_commit(pv_done);
       return true;
     };
-    for (int kt = 0; kt < ntk && ok; ++kt) {
-      const int s = kt & 1, use = kt >> 1;
-      if (!mbar_wait(&k_full[s], use & 1, abort_flag)) {
-        ok = false;
-        break;
+    for (int kt = 0; kt <= ntk && ok; ++kt) {
+      const int s = kt & 1;
+      if (kt < ntk) {
+        if (!mbar_wait(&k_full[s], (kt >> 1) & 1, abort_flag)) break;
+        fence_proxy_async_smem();
       }
-      if (kt >= 2 && !mbar_wait(&s_free[s], (use - 1) & 1, abort_flag)) {
-        ok = false;
-        break;
+      if (kt >= 1) {
+        if (!mbar_wait(&v_full[(kt - 1) & 1], ((kt - 1) >> 1) & 1, abort_flag)) break;
+        fence_proxy_async_smem();
       }
       tc_fence_after();
-      const uint32_t kb = k_s + s * L::kTileBytes;
+      for (int t = 0; t < ntiles && ok; ++t) {
+        if (kt >= 1) {
+          if (!issue_pv(t, kt - 1)) {
+            ok = false;
+            break;
+          }
+          if (t == ntiles - 1) umma_commit(&v_empty[(kt - 1) & 1]);
+        }
+        if (kt < ntk) {
+          const uint32_t kb = k_s + s * L::kTileBytes;
+          const uint32_t qb = q_s + t * L::kTileBytes;
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint64_t ad = umma_desc_sw128(q_s + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-        const uint64_t bd = umma_desc_sw128(kb + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-        umma_bf16_ss(tmem + s * 128, ad, bd, idesc_qk, k > 0 ? 1u : 0u);
+          for (int k = 0; k < D / 16; ++k) {
+            const uint64_t ad = umma_desc_sw128(qb + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+            const uint64_t bd = umma_desc_sw128(kb + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+            umma_bf16_ss(tmem + 128 * t, ad, bd, idesc_qk, k > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[t]);
+        }
       }
-      umma_commit(&k_empty[s]);
-      umma_commit(&s_full[s]);
-      if (kt >= 1 && !issue_pv(kt - 1)) ok = false;
+      if (ok && kt < ntk) umma_commit(&k_empty[s]);
     }
-    if (ok) issue_pv(ntk - 1);
+    if (ok) umma_commit(o_done);
     umma_commit(fin);
     mbar_wait_drain(fin, 0);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == 0) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -462,9 +463,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
 }
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s) {
-  // tiles per head <= ceil(N/128) + Cq (each group adds at most one ragged tile)
-  const long long tiles = (long long)(a.N + 127) / 128 + a.Cq;
-  dim3 grid((unsigned)tiles, a.BH);
+  // pairs of query tiles per head <= ceil(N/256) + Cq (one ragged pair per group)
+  const long long pairs = (long long)(a.N + 255) / 256 + a.Cq;
+  dim3 grid((unsigned)pairs, a.BH);
   if (a.d == 128) {
     const size_t sm = AttnSmem<128>::bytes();
     cudaError_t e =
