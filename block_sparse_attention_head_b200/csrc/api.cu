@@ -34,7 +34,7 @@ int check_params(const instagen_params* p) {
   if (!std::isfinite(p->exact_frac) || !std::isfinite(p->sample_frac) || p->exact_frac < 0.f ||
       p->sample_frac < 0.f)
     return IG_ERR_INVALID_ARG;
-  if (!std::isfinite(p->softmax_scale)) return IG_ERR_INVALID_ARG;
+  if (!std::isfinite(p->softmax_scale) || !(p->softmax_scale > 0.f)) return IG_ERR_INVALID_ARG;
   if (p->sampling != IG_SAMPLE_IMPORTANCE && p->sampling != IG_SAMPLE_UNIFORM) return IG_ERR_INVALID_ARG;
   return IG_OK;
 }

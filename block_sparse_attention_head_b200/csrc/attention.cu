@@ -224,56 +224,66 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
         cp_async_16(dst + (c >> 3) * 16384 + sw128_offset(rr, c & 7), src + c * 8, valid ? 16u : 0u);
     }
     cp_async_arrive_noinc(q_full);
+    // Warp w of the producer owns rows [64w, 64w+64) of every K/V tile; lane l
+    // resolves the permuted key positions of rows 64w+l and 64w+32+l (one tile
+    // ahead, since sample positions come from global memory).  The copies are
+    // issued lane -> 16-byte chunk of a row, so one warp instruction moves
+    // whole 256-byte rows (full L2 sectors).
+    const int pw = tp >> 5;
+    auto key_pos = [&](int j, int r) -> int {  // -1: padding slot
+      const int l = j * 128 + r;               // slot of tile row r in the key list
+      if (l < Xi) {
+        int lo = 0, hi = n_exact - 1;  // last e with gpre[e] <= l
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (gpre[mid] <= l)
+            lo = mid;
+          else
+            hi = mid - 1;
+        }
+        return gstart[lo] + (l - gpre[lo]);
+      }
+      if (l < Lk) return __ldg(spos + (l - Xi));
+      return -1;
+    };
+    auto checked = [&](int p) -> int {
+      if (p >= N) {
+        raise_error(kErrIndex);
+        return -1;
+      }
+      return p < 0 ? -1 : p;
+    };
+    constexpr int kCpr = D / 8;       // 16-byte chunks per row
+    constexpr int kRpi = 32 / kCpr;   // rows per warp instruction
+    const int rsub = lane / kCpr, ch = lane % kCpr;
+    // this lane's 16-byte chunk of rows i*kRpi + rsub (i = 0..64/kRpi-1) of the
+    // warp's 64 rows, from the row positions held by lanes (posA: rows 0-31,
+    // posB: rows 32-63)
+    const uint32_t lane_dst = (uint32_t)((ch >> 3) * 16384);
+    auto issue_rows = [&](const auto* base, uint32_t dst, int posA, int posB) {
+      const auto* head = base + (size_t)bh * N * D + ch * 8;
+#pragma unroll 4
+      for (int i = 0; i < 64 / kRpi; ++i) {
+        const int rl = i * kRpi + rsub;
+        const int p = __shfl_sync(0xffffffffu, i * kRpi < 32 ? posA : posB, rl & 31);
+        const int r = 64 * pw + rl;
+        cp_async_16(dst + lane_dst + sw128_offset(r, ch & 7), head + (size_t)(p < 0 ? 0 : p) * D,
+                    p < 0 ? 0u : 16u);
+      }
+    };
+    int nA = key_pos(0, 64 * pw + lane), nB = key_pos(0, 64 * pw + 32 + lane);
     for (int kt = 0; kt < ntk; ++kt) {
       const int s = kt & 1, use = kt >> 1;
-      int pos[2];
-      bool valid[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int l = kt * 128 + tp + h * kProducers;  // slot of this row in the key list
-        int p = -1;
-        if (l < Xi) {
-          int lo = 0, hi = n_exact - 1;  // last e with gpre[e] <= l
-          while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (gpre[mid] <= l)
-              lo = mid;
-            else
-              hi = mid - 1;
-          }
-          p = gstart[lo] + (l - gpre[lo]);
-        } else if (l < Lk) {
-          p = spos[l - Xi];
-        }
-        bool v = l < Lk;
-        if (v && (p < 0 || p >= N)) {
-          raise_error(kErrIndex);
-          v = false;
-        }
-        pos[h] = v ? p : 0;
-        valid[h] = v;
+      const int posA = checked(nA), posB = checked(nB);
+      if (kt + 1 < ntk) {
+        nA = key_pos(kt + 1, 64 * pw + lane);
+        nB = key_pos(kt + 1, 64 * pw + 32 + lane);
       }
       if (kt >= 2 && !mbar_wait(&k_empty[s], (use - 1) & 1, abort_flag)) break;
-      const uint32_t kdst = k_s + s * L::kTileBytes;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int r = tp + h * kProducers;
-        const __nv_bfloat16* ksrc = row_ptr(a.Kp, bh, N, pos[h], D);
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c)
-          cp_async_16(kdst + (c >> 3) * 16384 + sw128_offset(r, c & 7), ksrc + c * 8, valid[h] ? 16u : 0u);
-      }
+      issue_rows(a.Kp, k_s + s * L::kTileBytes, posA, posB);
       cp_async_arrive_noinc(&k_full[s]);
       if (kt >= 2 && !mbar_wait(&v_empty[s], (use - 1) & 1, abort_flag)) break;
-      const uint32_t vdst = v_s + s * L::kTileBytes;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int r = tp + h * kProducers;
-        const __half* vsrc = row_ptr(a.Vp, bh, N, pos[h], D);
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c)
-          cp_async_16(vdst + (c >> 3) * 16384 + sw128_offset(r, c & 7), vsrc + c * 8, valid[h] ? 16u : 0u);
-      }
+      issue_rows(a.Vp, v_s + s * L::kTileBytes, posA, posB);
       cp_async_arrive_noinc(&v_full[s]);
     }
     cp_async_wait_all();
@@ -288,42 +298,64 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
     float m_run = -__int_as_float(0x7f800000);
     float l_run = 0.f;
     bool ok = active;
-    for (int kt = 0; kt < ntk && ok; ++kt) {
-      // this warp's private copy of the tile's column log-weights (log2 units)
-      float* wb = bias_s + ((warp - 4) * 2 + (kt & 1)) * 128;
+    // column log-weights (log2 units) of key tile j, lane's 4 columns; loaded
+    // one tile ahead so the global-load latency stays off the critical path
+    auto load_bias = [&](int j, float* b) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int l = kt * 128 + lane * 4 + e;
-        float b;
+        const int l = j * 128 + lane * 4 + e;
         if (l < Xi)
-          b = 0.f;
+          b[e] = 0.f;
         else if (l < Lk)
-          b = sbias[l - Xi] * kLog2e;
+          b[e] = __ldg(sbias + (l - Xi));
         else
-          b = -__int_as_float(0x7f800000);
-        wb[lane * 4 + e] = b;
+          b[e] = -__int_as_float(0x7f800000);
       }
+    };
+    float bnext[4];
+    if (ok) load_bias(0, bnext);
+    for (int kt = 0; kt < ntk && ok; ++kt) {
+      // this warp's private copy of the tile's column log-weights
+      float* wb = bias_s + ((warp - 4) * 2 + (kt & 1)) * 128;
+      *reinterpret_cast<float4*>(wb + lane * 4) =
+          make_float4(bnext[0] * kLog2e, bnext[1] * kLog2e, bnext[2] * kLog2e, bnext[3] * kLog2e);
+      if (kt + 1 < ntk) load_bias(kt + 1, bnext);
       __syncwarp();
       if (!mbar_wait_warp(&s_full[t], kt & 1, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float4* b4 = reinterpret_cast<const float4*>(wb);
-      // pass 1: row maximum of the scaled, reweighted logits
-      float mx = -__int_as_float(0x7f800000);
-#pragma unroll 1
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float v[32];
-        tmem_ld32(s_col + c4 * 32, v);
-        tmem_wait_ld();
+      // the whole S row of this thread in registers: one TMEM round trip
+      float x[128];
+      tmem_ld32(s_col + 0, x);
+      tmem_ld32(s_col + 32, x + 32);
+      tmem_ld32(s_col + 64, x + 64);
+      tmem_ld32(s_col + 96, x + 96);
+      tmem_wait_ld();
+      // all-exact tiles carry no log-weight and no padding: scale after the max
+      const bool plain = kt * 128 + 128 <= Xi;
+      float mxp[4];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 bb = b4[(c4 * 32 + e) >> 2];
-          mx = fmaxf(mx, fmaxf(fmaxf(fmaf(v[e], a.scale_log2, bb.x), fmaf(v[e + 1], a.scale_log2, bb.y)),
-                               fmaxf(fmaf(v[e + 2], a.scale_log2, bb.z), fmaf(v[e + 3], a.scale_log2, bb.w))));
+      for (int e = 0; e < 4; ++e) mxp[e] = -__int_as_float(0x7f800000);
+      if (plain) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mxp[c & 3] = fmaxf(mxp[c & 3], x[c]);
+      } else {
+        const float4* b4 = reinterpret_cast<const float4*>(wb);
+#pragma unroll
+        for (int c = 0; c < 128; c += 4) {
+          const float4 bb = b4[c >> 2];
+          x[c + 0] = fmaf(x[c + 0], a.scale_log2, bb.x);
+          x[c + 1] = fmaf(x[c + 1], a.scale_log2, bb.y);
+          x[c + 2] = fmaf(x[c + 2], a.scale_log2, bb.z);
+          x[c + 3] = fmaf(x[c + 3], a.scale_log2, bb.w);
+          mxp[(c >> 2) & 1] = fmaxf(mxp[(c >> 2) & 1], fmaxf(x[c], x[c + 1]));
+          mxp[((c >> 2) & 1) + 2] = fmaxf(mxp[((c >> 2) & 1) + 2], fmaxf(x[c + 2], x[c + 3]));
         }
       }
+      float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
+      if (plain) mx *= a.scale_log2;  // scale > 0
       const float m_new = fmaxf(m_run, mx);
       const bool rescale = m_new > m_run + kRescaleThreshold;
       float alpha = 1.f;
@@ -331,8 +363,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
         alpha = ex2_approx(m_run - m_new);
         m_run = m_new;
       }
-      // O_t holds PV_t(kt-1) (the MMA pipe ran it before S_t(kt)); tcgen05.ld/st
-      // are warp-collective, so the warp rescales if any of its rows needs it
+      // P = 2^(x - m) as fp16 pairs into the first 64 columns of S_t (already
+      // read); the pairs are packed in place into slots of x already consumed
+      const float neg_m = -m_run;
+      float rsp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int c = c4 * 32 + e;
+          const float p0 = ex2_approx(plain ? fmaf(x[c], a.scale_log2, neg_m) : x[c] + neg_m);
+          const float p1 = ex2_approx(plain ? fmaf(x[c + 1], a.scale_log2, neg_m) : x[c + 1] + neg_m);
+          rsp[(e >> 1) & 3] += p0 + p1;
+          x[c4 * 16 + (e >> 1)] = __uint_as_float(pack_f16x2(p0, p1));
+        }
+        tmem_st16(s_col + c4 * 16, reinterpret_cast<const uint32_t*>(x + c4 * 16));
+      }
+      const float rs = (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
+      // O_t holds PV_t(kt-1) (the MMA pipe ran it before S_t(kt)) and PV_t(kt)
+      // waits for p_full; tcgen05.ld/st are warp-collective, so the warp
+      // rescales if any of its rows needs it (done after P so x is dead here)
       if (kt >= 1 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
         for (int c4 = 0; c4 < D / 32; ++c4) {
@@ -343,27 +393,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
           for (int e = 0; e < 32; ++e) o[e] *= alpha;
           tmem_st32(o_col + c4 * 32, o);
         }
-      }
-      // pass 2: P = 2^(x - m) as fp16 pairs into the first 64 columns of S_t
-      float rs = 0.f;
-#pragma unroll 1
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float v[32];
-        tmem_ld32(s_col + c4 * 32, v);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 bb = b4[(c4 * 32 + e) >> 2];
-          const float p0 = ex2_approx(fmaf(v[e], a.scale_log2, bb.x) - m_run);
-          const float p1 = ex2_approx(fmaf(v[e + 1], a.scale_log2, bb.y) - m_run);
-          const float p2 = ex2_approx(fmaf(v[e + 2], a.scale_log2, bb.z) - m_run);
-          const float p3 = ex2_approx(fmaf(v[e + 3], a.scale_log2, bb.w) - m_run);
-          rs += (p0 + p1) + (p2 + p3);
-          pk[e >> 1] = pack_f16x2(p0, p1);
-          pk[(e >> 1) + 1] = pack_f16x2(p2, p3);
-        }
-        tmem_st16(s_col + c4 * 16, pk);
       }
       tmem_wait_st();
       l_run = l_run * alpha + rs;

@@ -60,7 +60,7 @@ typedef struct {
   int32_t kmeans_iters;      /* Lloyd iterations (>= 1; 10 in every configuration) */
   float exact_frac;          /* exact share of keys: E = round(exact_frac * N)      */
   float sample_frac;         /* sampled share: m = round(sample_frac * N) draws      */
-  float softmax_scale;       /* logit scale, usually 1/sqrt(d)                       */
+  float softmax_scale;       /* logit scale > 0, usually 1/sqrt(d)                   */
   uint64_t seed;             /* Philox key                                           */
   uint32_t layer;            /* Philox counter word 3 (one stream per layer)         */
   int32_t sampling;          /* instagen_sampling                                    */
