@@ -42,6 +42,8 @@ def parse_args():
     ap.add_argument("--workload", default="wan2.1-14b_720p")
     ap.add_argument("--exact", type=float, default=None, help="override the exact share")
     ap.add_argument("--sample", type=float, default=None, help="override the sampled share")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the head count (same per-head shape; for profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
@@ -209,6 +211,9 @@ def main():
     args = parse_args()
     from block_sparse_attention_head_b200 import workloads
     w = workloads.WORKLOADS[args.workload]
+    if args.heads is not None:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.heads)
     exact = w.exact_frac if args.exact is None else args.exact
     sample = w.sample_frac if args.sample is None else args.sample
     if args.impl == "reference":
