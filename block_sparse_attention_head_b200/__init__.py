@@ -51,7 +51,8 @@ _lib = None
 _SYMBOLS = ("instagen_exact_budget", "instagen_sample_budget", "instagen_workspace_size",
             "instagen_cluster_workspace_size", "instagen_error_string", "instagen_device_status",
             "instagen_cluster", "instagen_permutation", "instagen_gather", "instagen_select_sample",
-            "instagen_attention", "instagen_forward", "instagen_forward_layout_get")
+            "instagen_attention", "instagen_forward", "instagen_forward_layout_get",
+            "instagen_cluster_static")
 
 
 def lib():
@@ -78,6 +79,7 @@ def lib():
         "instagen_attention": (ctypes.c_int, [PP, PP, PP, PP, PP, PP, PP, PP, PP, PP, P, PP, vp]),
         "instagen_forward": (ctypes.c_int, [PP, PP, PP, PP, P, PP, sz, vp]),
         "instagen_forward_layout_get": (ctypes.c_int, [P, ctypes.POINTER(ForwardLayout)]),
+        "instagen_cluster_static": (ctypes.c_int, [PP, i32, i32, PP, P, PP, PP, PP, PP, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -175,6 +177,24 @@ def cluster(X: torch.Tensor, C: int, iters: int, p: Params, init: Optional[torch
     ws = torch.empty(nws, dtype=torch.uint8, device=dev)
     _check(lib().instagen_cluster(_ptr(X), C, iters, _ptr(init), ctypes.byref(p), _ptr(cent), _ptr(assign),
                                   _ptr(perm), _ptr(offs), _ptr(ws), nws, _stream()), "instagen_cluster")
+    return cent, assign, perm, offs
+
+
+def cluster_static(X: torch.Tensor, C: int, iters: int, p: Params, init: Optional[torch.Tensor] = None):
+    """``cluster`` without a workspace: the scratch lives in a fixed device
+    array inside the library, for callers that may not allocate device
+    memory.  Only the outputs (allocated here by torch for convenience) are
+    passed; see ``instagen_cluster_static`` in include/instagen.h."""
+    _need(X, "X", torch.bfloat16, _bhnd(p))
+    dev = X.device
+    if init is not None:
+        _need(init, "init", torch.float32, (p.B, p.H, C, p.d))
+    cent = torch.empty((p.B, p.H, C, p.d), dtype=torch.float32, device=dev)
+    assign = torch.empty((p.B, p.H, p.N), dtype=torch.int32, device=dev)
+    perm = torch.empty_like(assign)
+    offs = torch.empty((p.B, p.H, C + 1), dtype=torch.int32, device=dev)
+    _check(lib().instagen_cluster_static(_ptr(X), C, iters, _ptr(init), ctypes.byref(p), _ptr(cent), _ptr(assign),
+                                         _ptr(perm), _ptr(offs), _stream()), "instagen_cluster_static")
     return cent, assign, perm, offs
 
 

@@ -5,3 +5,4 @@
 #include "select.cu"
 #include "attention.cu"
 #include "api.cu"
+#include "cluster_static.cu"

@@ -111,6 +111,34 @@ int instagen_cluster(const void* X, int32_t C, int32_t iters, const float* init,
                      size_t ws_bytes, void* stream);
 
 /*
+ * instagen_cluster without a workspace argument: the same k-means +
+ * permutation, with its scratch (centroid operand and norms) in a device
+ * array of INSTAGEN_CLUSTER_STATIC_SCRATCH_BYTES that the library itself
+ * owns.  No counterpart on the method's pages; this exists for callers that
+ * may not allocate device memory themselves -- plug-ins inside a host
+ * framework whose allocator owns all device memory, deployments that fix
+ * their memory budget at start-up and forbid later allocations, and code
+ * paths where a cudaMalloc would implicitly synchronise the device.
+ *   Arguments and outputs as instagen_cluster.  Nothing is allocated: no
+ *   cudaMalloc, cudaFree or allocating library routine is called.
+ *   Scratch needed = instagen_cluster_workspace_size(p, C); larger requests
+ *   return IG_ERR_WORKSPACE before anything is enqueued.  The scratch grows
+ *   with B*H, C and d but not with N: 16 MiB covers up to 63 heads at
+ *   C <= 512, d = 128 (e.g. the 40-head key clustering of Wan2.1-14B).
+ *   The array is held by every GPU that loads the library until the process
+ *   exits.  The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.
+ *   All calls share the one array and it keeps the last call's contents;
+ *   every element a call reads is written by the same call first, so nothing
+ *   needs clearing, but calls that overlap on the GPU (other streams, other
+ *   threads) race on it: serialise them.
+ */
+#define INSTAGEN_CLUSTER_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+int instagen_cluster_static(const void* X, int32_t C, int32_t iters, const float* init, const instagen_params* p,
+                            float* centroids, int32_t* assign, int32_t* perm, int32_t* offsets, void* stream);
+
+/*
  * Stable counting sort of given assignments (the permutation step alone).
  *   assign [B,H,N] int32 in [0, C); perm [B,H,N] out; offsets [B,H,C+1] out.
  * Out-of-range assignments are an IG_ERR_DEVICE_CHECK (the token is dropped).
