@@ -97,20 +97,18 @@ int run_cluster(const void* X, int C, int iters, const float* init, const instag
   const KmeansGeom g = ig::kmeans_geom(BH, p->N, p->d, C);
   if (!ws || ws_bytes < ig::kmeans_scratch_bytes(g) || (reinterpret_cast<uintptr_t>(ws) & 255u))
     return IG_ERR_WORKSPACE;
-  __nv_bfloat16* cmma = static_cast<__nv_bfloat16*>(ws);
-  float* norms = reinterpret_cast<float*>(static_cast<char*>(ws) +
-                                          align256((size_t)BH * g.c_pad * 2 * g.d * sizeof(__nv_bfloat16)));
+  const ig::KmeansScratch sc = ig::kmeans_scratch_carve(g, ws);
   CUtensorMap tx, tc;
   int rc = make_tmap_bf16(&tx, X, (uint64_t)BH * p->N, (uint64_t)p->d, 128);
   if (rc) return rc;
-  rc = make_tmap_bf16(&tc, cmma, (uint64_t)BH * g.c_pad, (uint64_t)2 * p->d, (uint32_t)g.chunk);
+  rc = make_tmap_bf16(&tc, sc.cmma, (uint64_t)BH * g.c_pad, (uint64_t)2 * p->d, (uint32_t)g.chunk);
   if (rc) return rc;
   const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
-  cudaError_t e = ig::launch_kmeans_init(g, Xb, init, cent, cmma, norms, s);
+  cudaError_t e = ig::launch_kmeans_init(g, Xb, init, cent, sc, s);
   for (int it = 0; it < iters && e == cudaSuccess; ++it) {
-    e = ig::launch_kmeans_assign(g, &tx, &tc, norms, assign, s);
+    e = ig::launch_kmeans_assign(g, &tx, &tc, sc.norms, assign, s);
     if (e == cudaSuccess) e = ig::launch_count_sort(assign, BH, p->N, C, perm, offsets, s);
-    if (e == cudaSuccess) e = ig::launch_kmeans_update(g, Xb, perm, offsets, cent, cmma, norms, s);
+    if (e == cudaSuccess) e = ig::launch_kmeans_update(g, Xb, perm, offsets, cent, sc, s);
   }
   return cuda_status(e);
 }

@@ -3,11 +3,12 @@
 // allocate device memory (see include/instagen.h).
 //
 // The scratch is the centroid operand of the distance GEMM ([BH, C_pad, 2d]
-// bf16) and the centroid norms ([BH, C_pad] fp32), the same layout
-// instagen_cluster carves from a caller-provided workspace.  Every element
-// the kernels read from it is first written by the same call (the init
-// kernel writes every row, padding included), so nothing has to be cleared
-// between calls; stale contents of an earlier call are never read.
+// bf16), the centroid norms ([BH, C_pad] fp32), the update's partial sums and
+// its arrival counters, the same layout instagen_cluster carves from a
+// caller-provided workspace.  Every element the kernels read from it is first
+// written by the same call (the init kernel writes every operand row, padding
+// included, and zeroes the counters), so nothing has to be cleared between
+// calls; stale contents of an earlier call are never read.
 #include "instagen.h"
 #include "internal.cuh"
 

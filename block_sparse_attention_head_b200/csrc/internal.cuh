@@ -18,15 +18,28 @@ struct KmeansGeom {
   int c_pad;   // C rounded up to a multiple of chunk
 };
 KmeansGeom kmeans_geom(int BH, int N, int d, int C);
+
+// Scratch of one clustering call, carved from one 256-byte aligned block:
+// the operand rows and norms above, fp32 partial sums of the clusters that
+// the update splits into several row pieces ([BH, part_slots, d]), and one
+// arrival counter per (head, cluster) ([BH, C] int32, zeroed by the init
+// kernel and returned to zero by the update that consumes it).
+struct KmeansScratch {
+  __nv_bfloat16* cmma;
+  float* norms;
+  float* partial;
+  int32_t* arrive;
+};
+int kmeans_part_slots(const KmeansGeom& g);
 size_t kmeans_scratch_bytes(const KmeansGeom& g);
+KmeansScratch kmeans_scratch_carve(const KmeansGeom& g, void* ws);
 
 cudaError_t launch_kmeans_init(const KmeansGeom& g, const __nv_bfloat16* X, const float* init, float* cent,
-                               __nv_bfloat16* cmma, float* norms, cudaStream_t s);
+                               const KmeansScratch& sc, cudaStream_t s);
 cudaError_t launch_kmeans_assign(const KmeansGeom& g, const CUtensorMap* tmap_x, const CUtensorMap* tmap_c,
                                  const float* norms, int32_t* assign, cudaStream_t s);
 cudaError_t launch_kmeans_update(const KmeansGeom& g, const __nv_bfloat16* X, const int32_t* perm,
-                                 const int32_t* offsets, float* cent, __nv_bfloat16* cmma, float* norms,
-                                 cudaStream_t s);
+                                 const int32_t* offsets, float* cent, const KmeansScratch& sc, cudaStream_t s);
 
 // ------------------------------------------------------- permutation/gather
 cudaError_t launch_count_sort(const int32_t* assign, int BH, int N, int C, int32_t* perm, int32_t* offsets,

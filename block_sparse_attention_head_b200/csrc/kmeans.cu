@@ -27,10 +27,38 @@ KmeansGeom kmeans_geom(int BH, int N, int d, int C) {
   return g;
 }
 
+// Rows summed by one CTA of the update; clusters with more members are split
+// into pieces of this many rows (in permuted order) whose partial sums are
+// added in piece order.
+constexpr int kUpdRows = 2048;
+
+// Partial-sum slots per head: the pieces of every cluster larger than one
+// piece.  A cluster of n > R rows has ceil(n/R) < 2n/R pieces, so all of them
+// together stay below 2N/R.
+int kmeans_part_slots(const KmeansGeom& g) { return (int)((2LL * g.N) / kUpdRows + 1); }
+
+namespace {
+size_t a256(size_t b) { return (b + 255) / 256 * 256; }
+}  // namespace
+
 size_t kmeans_scratch_bytes(const KmeansGeom& g) {
-  size_t cm = (size_t)g.BH * g.c_pad * 2 * g.d * sizeof(__nv_bfloat16);
-  size_t nm = (size_t)g.BH * g.c_pad * sizeof(float);
-  return ((cm + 255) / 256 * 256) + ((nm + 255) / 256 * 256);
+  const size_t BH = (size_t)g.BH;
+  return a256(BH * g.c_pad * 2 * g.d * sizeof(__nv_bfloat16)) + a256(BH * g.c_pad * sizeof(float)) +
+         a256(BH * kmeans_part_slots(g) * g.d * sizeof(float)) + a256(BH * g.C * sizeof(int32_t));
+}
+
+KmeansScratch kmeans_scratch_carve(const KmeansGeom& g, void* ws) {
+  const size_t BH = (size_t)g.BH;
+  char* b = static_cast<char*>(ws);
+  KmeansScratch sc;
+  sc.cmma = reinterpret_cast<__nv_bfloat16*>(b);
+  b += a256(BH * g.c_pad * 2 * g.d * sizeof(__nv_bfloat16));
+  sc.norms = reinterpret_cast<float*>(b);
+  b += a256(BH * g.c_pad * sizeof(float));
+  sc.partial = reinterpret_cast<float*>(b);
+  b += a256(BH * kmeans_part_slots(g) * g.d * sizeof(float));
+  sc.arrive = reinterpret_cast<int32_t*>(b);
+  return sc;
 }
 
 // Writes the hi/lo bf16 operand row and ||c||^2 for centroid row `c` (one warp).
@@ -53,12 +81,13 @@ __device__ __forceinline__ void write_operand_row(const float* c, int d, __nv_bf
 // One warp per (bh, padded centroid row).
 __global__ void kmeans_init_kernel(KmeansGeom g, const __nv_bfloat16* __restrict__ X, const float* __restrict__ init,
                                    float* __restrict__ cent, __nv_bfloat16* __restrict__ cmma,
-                                   float* __restrict__ norms) {
+                                   float* __restrict__ norms, int32_t* __restrict__ arrive) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int total = g.BH * g.c_pad;
   if (warp >= total) return;
   const int bh = warp / g.c_pad, j = warp % g.c_pad;
+  if (j < g.C && lane == 0) arrive[(size_t)bh * g.C + j] = 0;
   __nv_bfloat16* op = cmma + ((size_t)bh * g.c_pad + j) * 2 * g.d;
   if (j >= g.C) {  // padding row: zero operand, never selected
     for (int k = lane; k < 2 * g.d; k += 32) op[k] = __float2bfloat16_rn(0.f);
@@ -79,11 +108,11 @@ __global__ void kmeans_init_kernel(KmeansGeom g, const __nv_bfloat16* __restrict
 }
 
 cudaError_t launch_kmeans_init(const KmeansGeom& g, const __nv_bfloat16* X, const float* init, float* cent,
-                               __nv_bfloat16* cmma, float* norms, cudaStream_t s) {
+                               const KmeansScratch& sc, cudaStream_t s) {
   const long long warps = (long long)g.BH * g.c_pad;
   const int threads = 256;
   const long long blocks = (warps * 32 + threads - 1) / threads;
-  kmeans_init_kernel<<<(unsigned)blocks, threads, 0, s>>>(g, X, init, cent, cmma, norms);
+  kmeans_init_kernel<<<(unsigned)blocks, threads, 0, s>>>(g, X, init, cent, sc.cmma, sc.norms, sc.arrive);
   return cudaGetLastError();
 }
 
@@ -308,52 +337,153 @@ cudaError_t launch_kmeans_assign(const KmeansGeom& g, const CUtensorMap* tmap_x,
 }
 
 // ------------------------------------------------------------------ update
-// One CTA per (cluster, head).  Members are read in permuted (stable) order by
-// kUpdSlots row slots; each slot sums a fixed subsequence of rows and the slot
-// sums are added in slot order, so the result does not depend on scheduling.
+// A grid over row pieces: a cluster of n members gets ceil(n/R) pieces of at
+// most R = kUpdRows consecutive permuted rows (an empty cluster one empty
+// piece), so the work of a CTA stays bounded however skewed the cluster sizes
+// are.  A CTA finds its (cluster, piece) by a scan over the cluster sizes and
+// sums its rows in kUpdThreads / (d/8) row slots, each slot a fixed
+// subsequence of rows, the slot sums added in slot order.  A single-piece
+// cluster writes its mean at once (an empty one keeps its centroid); the
+// pieces of a larger cluster store their sums, and the CTA that arrives last
+// adds them in piece order and writes the mean.  Every sum runs in a fixed
+// order, so the centroids do not depend on scheduling.
 constexpr int kUpdThreads = 256;
+constexpr int kUpdUnroll = 4;  // rows in flight per slot
+
+__device__ __forceinline__ int update_pieces(int n) { return n <= kUpdRows ? 1 : (n + kUpdRows - 1) / kUpdRows; }
 
 __global__ void __launch_bounds__(kUpdThreads)
     kmeans_update_kernel(KmeansGeom g, const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ perm,
                          const int32_t* __restrict__ offsets, float* __restrict__ cent,
-                         __nv_bfloat16* __restrict__ cmma, float* __restrict__ norms) {
+                         __nv_bfloat16* __restrict__ cmma, float* __restrict__ norms, float* __restrict__ partial,
+                         int32_t* __restrict__ arrive, int part_slots) {
   __shared__ float part[kUpdThreads * 8];
   __shared__ float red[32];
-  const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-  const int cpr = g.d / 8;             // 16-byte chunks per row
+  __shared__ int scan_np[kUpdThreads / 32], scan_mp[kUpdThreads / 32];
+  __shared__ int s_c, s_piece, s_np, s_base, s_last;
+  const int bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int32_t* off = offsets + (size_t)bh * (g.C + 1);
+
+  // (cluster, piece) of this CTA: exclusive scans over the clusters of the
+  // piece count and of the pieces that belong to multi-piece clusters
+  const int per = (g.C + kUpdThreads - 1) / kUpdThreads;
+  const int c0 = min(tid * per, g.C), c1 = min(c0 + per, g.C);
+  int np_own = 0, mp_own = 0;
+  for (int c = c0; c < c1; ++c) {
+    const int k = update_pieces(max(off[c + 1] - off[c], 0));
+    np_own += k;
+    if (k > 1) mp_own += k;
+  }
+  int np_inc = np_own, mp_inc = mp_own;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, np_inc, o);
+    const int b = __shfl_up_sync(0xffffffffu, mp_inc, o);
+    if (lane >= o) {
+      np_inc += a;
+      mp_inc += b;
+    }
+  }
+  if (lane == 31) {
+    scan_np[wid] = np_inc;
+    scan_mp[wid] = mp_inc;
+  }
+  if (tid == 0) s_c = -1;
+  __syncthreads();
+  int at = np_inc - np_own, mb = mp_inc - mp_own;
+  for (int w = 0; w < wid; ++w) {
+    at += scan_np[w];
+    mb += scan_mp[w];
+  }
+  const int t = blockIdx.x;
+  if (t >= at && t < at + np_own) {
+    for (int c = c0; c < c1; ++c) {
+      const int k = update_pieces(max(off[c + 1] - off[c], 0));
+      if (t < at + k) {
+        s_c = c;
+        s_piece = t - at;
+        s_np = k;
+        s_base = mb;
+        break;
+      }
+      at += k;
+      if (k > 1) mb += k;
+    }
+  }
+  __syncthreads();
+  const int c = s_c;
+  if (c < 0) return;  // past the last piece of this head
+  const int piece = s_piece, npieces = s_np;
+  if (npieces > 1 && s_base + npieces > part_slots) {  // offsets that do not sum to N
+    if (tid == 0) raise_error(kErrIndex);
+    return;
+  }
+
+  const int cpr = g.d / 8;  // 16-byte chunks per row
   const int slots = kUpdThreads / cpr;
   const int slot = tid / cpr, ch = tid % cpr;
-  const int lo = offsets[(size_t)bh * (g.C + 1) + c];
-  const int hi = offsets[(size_t)bh * (g.C + 1) + c + 1];
+  const int lo = off[c], hi = off[c + 1];
+  const int plo = lo + piece * kUpdRows, phi = min(hi, plo + kUpdRows);
+  const int32_t* prow = perm + (size_t)bh * g.N;
+  const __nv_bfloat16* xh = X + (size_t)bh * g.N * g.d + ch * 8;
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  for (int p = lo + slot; p < hi; p += slots) {
-    const int src = perm[(size_t)bh * g.N + p];
-    if (src < 0 || src >= g.N) {
-      raise_error(kErrIndex);
-      continue;
-    }
-    const uint4 raw = *reinterpret_cast<const uint4*>(X + ((size_t)bh * g.N + src) * g.d + ch * 8);
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+  for (int p0 = plo + slot; p0 < phi; p0 += kUpdUnroll * slots) {
+    int src[kUpdUnroll];
+    uint4 raw[kUpdUnroll];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __bfloat1622float2(h2[e]);
-      acc[2 * e] += f.x;
-      acc[2 * e + 1] += f.y;
+    for (int u = 0; u < kUpdUnroll; ++u) {
+      const int p = p0 + u * slots;
+      src[u] = p < phi ? prow[p] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kUpdUnroll; ++u) {
+      const bool live = p0 + u * slots < phi;
+      const bool ok = src[u] >= 0 && src[u] < g.N;
+      if (live && !ok) raise_error(kErrIndex);
+      raw[u] = (live && ok) ? *reinterpret_cast<const uint4*>(xh + (size_t)src[u] * g.d) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kUpdUnroll; ++u) {  // rows added in permuted order
+      if (p0 + u * slots >= phi) break;
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h2[e]);
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
+      }
     }
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) part[slot * g.d + ch * 8 + e] = acc[e];
   __syncthreads();
+  float sum = 0.f;
+  if (tid < g.d)
+    for (int sl = 0; sl < slots; ++sl) sum += part[sl * g.d + tid];
+
+  if (npieces > 1) {
+    float* pbase = partial + ((size_t)bh * part_slots + s_base) * g.d;
+    if (tid < g.d) pbase[(size_t)piece * g.d + tid] = sum;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(&arrive[(size_t)bh * g.C + c], 1) == npieces - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (tid < g.d) {
+      sum = 0.f;
+      for (int q = 0; q < npieces; ++q) sum += __ldcg(pbase + (size_t)q * g.d + tid);
+    }
+    if (tid == 0) arrive[(size_t)bh * g.C + c] = 0;  // ready for the next update
+  }
+
   const int n = hi - lo;
   float sq = 0.f;
   if (tid < g.d) {
     float* cr = cent + ((size_t)bh * g.C + c) * g.d;
     float v;
     if (n > 0) {
-      float sum = 0.f;
-      for (int sl = 0; sl < slots; ++sl) sum += part[sl * g.d + tid];
       v = sum / (float)n;
       cr[tid] = v;
     } else {
@@ -368,7 +498,7 @@ __global__ void __launch_bounds__(kUpdThreads)
   }
   // ||c||^2: warp sums then a fixed-order sum of the warp partials
   for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-  if ((tid & 31) == 0) red[tid >> 5] = sq;
+  if (lane == 0) red[wid] = sq;
   __syncthreads();
   if (tid == 0) {
     float tot = 0.f;
@@ -378,10 +508,12 @@ __global__ void __launch_bounds__(kUpdThreads)
 }
 
 cudaError_t launch_kmeans_update(const KmeansGeom& g, const __nv_bfloat16* X, const int32_t* perm,
-                                 const int32_t* offsets, float* cent, __nv_bfloat16* cmma, float* norms,
-                                 cudaStream_t s) {
-  dim3 grid(g.C, g.BH);
-  kmeans_update_kernel<<<grid, kUpdThreads, 0, s>>>(g, X, perm, offsets, cent, cmma, norms);
+                                 const int32_t* offsets, float* cent, const KmeansScratch& sc, cudaStream_t s) {
+  // at most C + N/R pieces per head (every cluster adds at most one piece
+  // beyond n/R); CTAs past a head's last piece return at once
+  dim3 grid(g.C + (g.N + kUpdRows - 1) / kUpdRows, g.BH);
+  kmeans_update_kernel<<<grid, kUpdThreads, 0, s>>>(g, X, perm, offsets, cent, sc.cmma, sc.norms, sc.partial,
+                                                     sc.arrive, kmeans_part_slots(g));
   return cudaGetLastError();
 }
 

@@ -6,44 +6,80 @@
 #include "internal.cuh"
 #include "ptx.cuh"
 
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 namespace ig {
 
 // --------------------------------------------------------- counting sort
-// One CTA per head.  Warp w owns a contiguous segment of the tokens; phase 1
-// counts its segment per cluster, phase 2 turns the (cluster-major,
-// warp-minor) counts into write cursors, phase 3 walks each segment in order
-// (32 tokens at a time, ranks inside a step from __match_any_sync) so equal
-// clusters keep ascending token index.
+// One thread-block cluster of S CTAs per head (S <= 8); CTA r owns the r-th
+// of S contiguous token ranges, and warp w of it a contiguous sub-range.
+// Phase 1 counts every warp's range per cluster; the CTA totals are exchanged
+// through distributed shared memory, giving every CTA the global cluster
+// starts and the number of earlier tokens of each cluster in lower-ranked
+// CTAs; phase 3 walks each warp range in order (32 tokens at a time, ranks
+// inside a step from __match_any_sync), so equal clusters keep ascending
+// token index.  The sort is a single launch and needs no global scratch.
+constexpr int kSortMaxCtas = 8;
+constexpr int kSortUnroll = 4;
+
 __global__ void count_sort_kernel(const int32_t* __restrict__ assign, int N, int C, int32_t* __restrict__ perm,
                                   int32_t* __restrict__ offsets) {
-  extern __shared__ int cnt[];  // [nwarps][C] counters, then C+1 cluster offsets
+  extern __shared__ int sort_smem[];  // cnt [nwarps][C], ctot [C], before [C], base [C+1]
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int S = (int)cluster.num_blocks();
+  const int r = (int)cluster.block_rank();
   const int nwarps = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
+  const int bh = blockIdx.y;
   const int32_t* a = assign + (size_t)bh * N;
-  int* base = cnt + nwarps * C;
+  int* cnt = sort_smem;
+  int* ctot = cnt + nwarps * C;
+  int* before = ctot + C;
+  int* base = before + C;
   for (int i = threadIdx.x; i < nwarps * C; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
-  const int seg = (N + nwarps - 1) / nwarps;
-  const int s0 = min(N, warp * seg), s1 = min(N, s0 + seg);
-  for (int i = s0 + lane; i < s1; i += 32) {
-    const int c = a[i];
-    if (c >= 0 && c < C)
-      atomicAdd(&cnt[warp * C + c], 1);
-    else
-      raise_error(kErrIndex);
+  const int q0 = (int)((long long)N * r / S), q1 = (int)((long long)N * (r + 1) / S);
+  const int seg = (q1 - q0 + nwarps - 1) / nwarps;
+  const int s0 = min(q1, q0 + warp * seg), s1 = min(q1, s0 + seg);
+  for (int i0 = s0 + lane; i0 < s1; i0 += 32 * kSortUnroll) {
+    int v[kSortUnroll];
+#pragma unroll
+    for (int u = 0; u < kSortUnroll; ++u) v[u] = (i0 + 32 * u < s1) ? a[i0 + 32 * u] : 0;
+#pragma unroll
+    for (int u = 0; u < kSortUnroll; ++u) {
+      if (i0 + 32 * u >= s1) break;
+      if (v[u] >= 0 && v[u] < C)
+        atomicAdd(&cnt[warp * C + v[u]], 1);
+      else
+        raise_error(kErrIndex);
+    }
   }
   __syncthreads();
-  // cluster totals and their exclusive prefix (one warp, sequential over chunks of 32)
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    int t = 0;
+    for (int w = 0; w < nwarps; ++w) t += cnt[w * C + c];
+    ctot[c] = t;
+  }
+  cluster.sync();  // every CTA's totals visible to the cluster
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    int all = 0, bef = 0;
+    for (int q = 0; q < S; ++q) {
+      const int v = cluster.map_shared_rank(ctot, q)[c];
+      all += v;
+      if (q < r) bef += v;
+    }
+    base[c] = all;
+    before[c] = bef;
+  }
+  cluster.sync();  // no remote reads after this point
+  // exclusive prefix of the cluster totals (one warp, chunks of 32)
   if (warp == 0) {
     int run = 0;
     for (int c0 = 0; c0 < C; c0 += 32) {
       const int c = c0 + lane;
-      int tot = 0;
-      if (c < C)
-        for (int w = 0; w < nwarps; ++w) tot += cnt[w * C + c];
+      const int tot = c < C ? base[c] : 0;
       int incl = tot;
       for (int o = 1; o < 32; o <<= 1) {
         const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -55,9 +91,10 @@ __global__ void count_sort_kernel(const int32_t* __restrict__ assign, int N, int
     if (lane == 0) base[C] = run;
   }
   __syncthreads();
-  for (int c = threadIdx.x; c <= C; c += blockDim.x) offsets[(size_t)bh * (C + 1) + c] = base[c];
+  if (r == 0)
+    for (int c = threadIdx.x; c <= C; c += blockDim.x) offsets[(size_t)bh * (C + 1) + c] = base[c];
   for (int c = threadIdx.x; c < C; c += blockDim.x) {
-    int run = base[c];
+    int run = base[c] + before[c];
     for (int w = 0; w < nwarps; ++w) {
       const int t = cnt[w * C + c];
       cnt[w * C + c] = run;
@@ -66,10 +103,12 @@ __global__ void count_sort_kernel(const int32_t* __restrict__ assign, int N, int
   }
   __syncthreads();
   const unsigned lt_mask = (1u << lane) - 1u;
+  int nxt = (s0 + lane < s1) ? a[s0 + lane] : -1;
   for (int i0 = s0; i0 < s1; i0 += 32) {
     const int i = i0 + lane;
-    int c = (i < s1) ? a[i] : -1;
-    if (c >= C) c = -1;
+    int c = nxt;
+    nxt = (i + 32 < s1) ? a[i + 32] : -1;  // next step's load in flight
+    if (c >= C || c < 0) c = -1;
     const unsigned same = __match_any_sync(0xffffffffu, c);
     const int rank = __popc(same & lt_mask);
     int pos = 0;
@@ -83,14 +122,28 @@ __global__ void count_sort_kernel(const int32_t* __restrict__ assign, int N, int
 
 cudaError_t launch_count_sort(const int32_t* assign, int BH, int N, int C, int32_t* perm, int32_t* offsets,
                               cudaStream_t s) {
-  // as many warps (<= 32) as fit 160 KB of per-warp counters
+  // one CTA per 4096 tokens of a head, up to a cluster of 8; as many warps
+  // (<= 32) as fit 160 KB of per-warp counters
+  int S = (N + 4095) / 4096;
+  S = S < 1 ? 1 : (S > kSortMaxCtas ? kSortMaxCtas : S);
   int nwarps = (int)((160 * 1024) / ((size_t)C * 4));
   nwarps = nwarps < 1 ? 1 : (nwarps > 32 ? 32 : nwarps);
-  const size_t sm = ((size_t)nwarps * C + C + 1) * sizeof(int);
+  const size_t sm = ((size_t)nwarps * C + 3 * (size_t)C + 1) * sizeof(int);
   cudaError_t e = cudaFuncSetAttribute(count_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
-  count_sort_kernel<<<BH, nwarps * 32, sm, s>>>(assign, N, C, perm, offsets);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S, BH);
+  cfg.blockDim = dim3(nwarps * 32);
+  cfg.dynamicSmemBytes = sm;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, count_sort_kernel, assign, N, C, perm, offsets);
 }
 
 // ---------------------------------------------------------------- gather

@@ -104,7 +104,9 @@ def test_permutation_bit_exact(oracle_runs, case):
 
 def test_permutation_edge_cases():
     # all tokens in one cluster, clusters left empty, single token
-    for N, C, fill in ((333, 5, "one"), (1000, 64, "random"), (1, 3, "one")):
+    # (the last two span a cluster of 8 CTAs, one with every token in one cluster)
+    for N, C, fill in ((333, 5, "one"), (1000, 64, "random"), (1, 3, "one"), (70001, 500, "random"),
+                       (50000, 7, "one")):
         p = ig.make_params(1, 1, N, 64, C, C)
         a = np.full(N, 2 % C, np.int32) if fill == "one" else np.random.default_rng(N).integers(0, C // 2, N)
         perm, offs = ig.permutation(cuda(a.astype(np.int32)[None, None]), C, p)
@@ -191,6 +193,33 @@ def test_kmeans_one_step_matches_oracle(oracle_mod, oracle_runs, case):
             np.testing.assert_allclose(np_(cent)[0, h][same], ref[same], rtol=0, atol=2e-4)
             # the returned permutation is the stable sort of the returned assignment
             assert np.array_equal(np_(perm)[0, h], np.argsort(ga[h], kind="stable"))
+    ig.device_status()
+
+
+@pytest.mark.parametrize("iters", [1, 3])
+def test_kmeans_large_clusters(oracle_mod, iters):
+    """Clusters of ~10k members, which the centroid update splits into pieces
+    of 2048 rows whose partial sums are added in piece order by the last piece
+    to finish; 3 iterations check that the per-cluster arrival counters are
+    ready again for the next update.  The counting sort spans 8 CTAs."""
+    H, N, d, C = 2, 30001, 128, 5
+    Q, K, V = workloads.random_small(31, N, d, n_centres=3, sigma=0.4, H=H)
+    p = ig.make_params(1, H, N, d, C, C, iters=iters)
+    Xn = [np_(K[0, h].float()) for h in range(H)]
+    init = np.stack([oracle_mod.kmeans_init(x, C) for x in Xn])[None]
+    cent, assign, perm, offs = ig.cluster(K.cuda(), C, iters, p, init=cuda(init))
+    ga, gc = np_(assign)[0], np_(cent)[0]
+    assert np.bincount(ga.ravel(), minlength=C).max() > 4 * 2048
+    for h in range(H):
+        if iters == 1:
+            oa, _ = oracle_mod.kmeans_assign(Xn[h], init[0, h])
+            assert np.mean(ga[h] == oa) >= 0.999
+        x = Xn[h].astype(np.float64)
+        for j in range(C):
+            if np.any(ga[h] == j):
+                np.testing.assert_allclose(gc[h, j], x[ga[h] == j].mean(0), rtol=0, atol=2e-4)
+        assert np.array_equal(np_(perm)[0, h], np.argsort(ga[h], kind="stable"))
+        assert np.array_equal(np_(offs)[0, h], np.concatenate([[0], np.cumsum(np.bincount(ga[h], minlength=C))]))
     ig.device_status()
 
 
@@ -316,10 +345,17 @@ def test_full_size_heads_sampled_parity(oracle_mod):
     # k-means step from the oracle's init (= the default init)
     for X, C, attr in ((Q, w.Cq, "q_assign"), (K, w.Ck, "k_assign")):
         cent, assign, _, _ = ig.cluster(X.cuda(), C, 1, p)
-        ga = np_(assign)[0]
+        ga, gc = np_(assign)[0], np_(cent)[0]
         for h in range(H):
             agree = np.mean(ga[h] == getattr(hr[h], attr))
             assert agree >= 0.999, f"C={C} head {h}: {agree}"
+            # the updated centroids are the means of the returned clusters
+            x = np_(X[0, h].float()).astype(np.float64)
+            sums = np.zeros((C, w.d))
+            np.add.at(sums, ga[h], x)
+            n = np.bincount(ga[h], minlength=C)
+            live = n > 0
+            np.testing.assert_allclose(gc[h][live], sums[live] / n[live, None], rtol=0, atol=2e-4)
     # select / sample from the oracle's centroids
     eg, cnt, sp, sb = ig.select_sample(_stack(hr, "cq"), _stack(hr, "ck"), _stack(hr, "k_offsets"), p)
     for h in range(H):
