@@ -14,7 +14,7 @@ namespace ig {
 // bf16(c - hi) ("lo"); norms [BH, c_pad] fp32 = ||c||^2 of the fp32 centroid.
 struct KmeansGeom {
   int BH, N, d, C;
-  int chunk;   // centroids per MMA chunk (multiple of 16, <= 128)
+  int chunk;   // centroids per MMA chunk (multiple of 16, <= 256)
   int c_pad;   // C rounded up to a multiple of chunk
 };
 KmeansGeom kmeans_geom(int BH, int N, int d, int C);

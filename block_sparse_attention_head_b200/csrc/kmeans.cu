@@ -21,9 +21,12 @@ KmeansGeom kmeans_geom(int BH, int N, int d, int C) {
   g.N = N;
   g.d = d;
   g.C = C;
-  int c16 = (C + 15) / 16 * 16;
-  g.chunk = c16 < 128 ? c16 : 128;
-  g.c_pad = (C + g.chunk - 1) / g.chunk * g.chunk;
+  // chunks of <= 256 centroids (one MMA's N), as few and as even as possible,
+  // each a multiple of 16 so that each CTA of a pair holds whole 8-row groups
+  const int c16 = (C + 15) / 16 * 16;
+  const int nch = (c16 + 255) / 256;
+  g.chunk = ((c16 + nch - 1) / nch + 15) / 16 * 16;
+  g.c_pad = nch * g.chunk;
   return g;
 }
 
@@ -89,9 +92,9 @@ __global__ void kmeans_init_kernel(KmeansGeom g, const __nv_bfloat16* __restrict
   const int bh = warp / g.c_pad, j = warp % g.c_pad;
   if (j < g.C && lane == 0) arrive[(size_t)bh * g.C + j] = 0;
   __nv_bfloat16* op = cmma + ((size_t)bh * g.c_pad + j) * 2 * g.d;
-  if (j >= g.C) {  // padding row: zero operand, never selected
+  if (j >= g.C) {  // padding row: zero operand, infinite norm, never selected
     for (int k = lane; k < 2 * g.d; k += 32) op[k] = __float2bfloat16_rn(0.f);
-    if (lane == 0) norms[(size_t)bh * g.c_pad + j] = 0.f;
+    if (lane == 0) norms[(size_t)bh * g.c_pad + j] = __int_as_float(0x7f800000);
     return;
   }
   float* c = cent + ((size_t)bh * g.C + j) * g.d;
@@ -117,32 +120,82 @@ cudaError_t launch_kmeans_init(const KmeansGeom& g, const __nv_bfloat16* X, cons
 }
 
 // ------------------------------------------------------------------ assign
-// CTA = up to kPairsPerCta pairs of 128-token tiles of one head (M = 2 x 128),
-// streaming the head's centroid operand through shared memory in K-blocks of
-// 64 columns (TMA, 128-byte swizzle) for each chunk of <= 128 centroids.
-// TMEM: 2 buffers x 2 tiles x 128 fp32 columns; the epilogue of chunk c
-// (argmin over the chunk's columns) overlaps the MMAs of chunk c+1.
-// Warps: 0 TMA producer, 1 MMA issuer (+ TMEM owner), 4-7 epilogue tile 0,
-// 8-11 epilogue tile 1; warps 2-3 only join the block-wide barriers.
+// CTA pairs: a cluster of two CTAs (the two SMs of a TPC) computes the
+// distances of a unit of 256 tokens of one head to a chunk of <= 256
+// centroids, one M = 256 tcgen05 MMA (.cta_group::2) per K-step of 16.  Each
+// CTA stages its 128 token rows and half of the chunk's centroid rows and
+// receives its rows' fp32 products in its own TMEM.  Few large MMAs matter
+// here: M = 128 or N = 128 MMAs leave the tensor pipe half idle on issue and
+// shared-memory reads, while one M = 256, N = 256 MMA per K-step keeps it
+// busy.  Persistent: the pairs walk contiguous ranges of units over all
+// heads.  Token tiles are double-buffered (the next unit streams in from HBM
+// during the current one) and the centroid halves stream through a ring of
+// K-blocks of 64 columns (TMA, 128-byte swizzle).  TMEM: 2 buffers x 256 fp32
+// columns; epilogue group b (4 warps) reduces the chunks that land in buffer
+// b, and the two groups' partial minima of a unit are merged through shared
+// memory.  Warps: 0 centroid producer, 1 TMEM owner + MMA issuer (leader
+// CTA), 2 token producer, 4-7 / 8-11 epilogue groups 0 / 1.
 namespace {
 constexpr int kAssignThreads = 384;
-constexpr int kAssignStages = 4;
-constexpr int kPairsPerCta = 4;
+constexpr int kAssignStages = 6;
+constexpr int kAssignXBufs = 3;  // token tiles in flight
 
 template <int D>
 struct AssignSmem {
-  static constexpr int kXBlocks = D / 64;                 // 64-column K-blocks of a token tile
+  static constexpr int kXBlocks = D / 64;                   // 64-column K-blocks of a token tile
   static constexpr int kXTileBytes = kXBlocks * 128 * 128;  // 128 rows x D bf16
-  static constexpr int kStageBytes = 128 * 128;           // <= 128 centroid rows x 64 columns
-  static constexpr int kX = 0;
-  static constexpr int kStages = kX + 2 * kXTileBytes;
-  static constexpr int kBars = kStages + kAssignStages * kStageBytes;
-  static constexpr int kNumBars = 2 * kAssignStages + 2 + 2 + 2 + 1;  // c_full, c_empty, x_full, x_empty, t_full, t_empty, fin
-  static constexpr int kMisc = kBars + kNumBars * 8;            // tmem base, abort flag
-  static constexpr int kNorms = kMisc + 16;
-  static size_t bytes(int c_pad) { return 1024 + kNorms + (size_t)c_pad * 4; }
+  static constexpr int kStageBytes = 128 * 128;             // <= 128 centroid rows x 64 columns
+  static constexpr int kX = 0;                              // token tile ring
+  static constexpr int kStages = kX + kAssignXBufs * kXTileBytes;
+  static constexpr int kMerge = kStages + kAssignStages * kStageBytes;  // [2 slots][128] (distance, index)
+  static constexpr int kNorms = kMerge + 2 * 128 * 8;                   // [8 epilogue warps][256] fp32
+  static constexpr int kBars = kNorms + 8 * 256 * 4;
+  // c_full, c_empty [stages]; x_full, x_empty [x bufs]; t_full, t_empty, m_full, m_empty [2]; fin
+  static constexpr int kNumBars = 2 * kAssignStages + 2 * kAssignXBufs + 8 + 1;
+  static constexpr int kMisc = kBars + kNumBars * 8;  // tmem base, abort flag
+  static constexpr size_t bytes() { return 1024 + kMisc + 16; }
 };
 }  // namespace
+
+// Folds 32 distance columns into the running (best, best_j): dist =
+// ||c||^2 - 2 x.c with the norms `nw` (shared memory, same address in every
+// lane); columns at or past `chunk` are ignored.  Argmin by a pairwise tree in
+// which the right operand wins only when strictly smaller, so ties keep the
+// lowest index; padding centroids have an infinite norm and never win.
+__device__ __forceinline__ void assign_reduce32(float (&x)[32], const float4* nw, int cb, int chunk, int j0,
+                                                float& best, int& best_j) {
+  float4 nv[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) nv[u] = nw[u];
+  const float* nf = reinterpret_cast<const float*>(nv);
+  if (cb + 32 > chunk) {  // columns past the chunk hold no product
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (cb + e >= chunk) x[e] = 0.f;
+  }
+  float m[16];
+  int ix[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float a = fmaf(-2.f, x[2 * k], nf[2 * k]);
+    const float b = fmaf(-2.f, x[2 * k + 1], nf[2 * k + 1]);
+    ix[k] = b < a ? 2 * k + 1 : 2 * k;
+    m[k] = fminf(a, b);
+  }
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+    for (int k = 0; k < w; ++k) {
+      const bool lt = m[2 * k + 1] < m[2 * k];
+      ix[k] = lt ? ix[2 * k + 1] : ix[2 * k];
+      m[k] = fminf(m[2 * k], m[2 * k + 1]);
+    }
+  }
+  if (m[0] < best) {
+    best = m[0];
+    best_j = j0 + ix[0];
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kAssignThreads, 1)
@@ -152,188 +205,255 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
-  uint64_t* c_full = bars;
+  uint64_t* c_full = bars;  // leader's copy counts both CTAs' bytes
   uint64_t* c_empty = bars + kAssignStages;
-  uint64_t* x_full = bars + 2 * kAssignStages;
-  uint64_t* x_empty = x_full + 1;
-  uint64_t* t_full = x_full + 2;   // [2] per TMEM buffer
-  uint64_t* t_empty = x_full + 4;  // [2]
-  uint64_t* fin = x_full + 6;
+  uint64_t* x_full = bars + 2 * kAssignStages;  // [x bufs] leader's copy counts both CTAs' bytes
+  uint64_t* x_empty = x_full + kAssignXBufs;    // [x bufs]
+  uint64_t* t_full = x_empty + kAssignXBufs;    // [2] per TMEM buffer
+  uint64_t* t_empty = t_full + 2;               // [2] leader's copy, both CTAs' epilogue warps
+  uint64_t* m_full = t_full + 4;                // [2] per merge slot
+  uint64_t* m_empty = t_full + 6;               // [2]
+  uint64_t* fin = t_full + 8;
+  float2* merge = reinterpret_cast<float2*>(smem + L::kMerge);
+  float4* norms_s = reinterpret_cast<float4*>(smem + L::kNorms);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-  float* norm_s = reinterpret_cast<float*>(smem + L::kNorms);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.y;
-  const int pairs_total = (g.N + 255) / 256;
-  const int pair0 = blockIdx.x * kPairsPerCta;
-  const int npairs = min(kPairsPerCta, pairs_total - pair0);
-  if (npairs <= 0) return;
+  const uint32_t rank = cluster_ctarank();
+  const int uph = (g.N + 255) / 256;  // 256-token units per head
+  const long long total = (long long)g.BH * uph;
+  const int npairs = gridDim.x / 2, pair = blockIdx.x / 2;
+  const long long u0 = total * pair / npairs;
+  const int nunits = (int)(total * (pair + 1) / npairs - u0);
+  if (nunits <= 0) return;  // the same for both CTAs of the pair
   const int nchunks = g.c_pad / g.chunk;
+  const int half = g.chunk / 2;         // centroid rows per CTA per chunk
   const int kblocks = 2 * L::kXBlocks;  // hi blocks then lo blocks
 
-  for (int j = tid; j < g.c_pad; j += blockDim.x) norm_s[j] = norms[(size_t)bh * g.c_pad + j];
   if (tid == 0) {
     for (int s = 0; s < kAssignStages; ++s) {
       mbar_init(&c_full[s], 1);
       mbar_init(&c_empty[s], 1);
     }
-    mbar_init(x_full, 1);
-    mbar_init(x_empty, 1);
+    for (int b = 0; b < kAssignXBufs; ++b) {
+      mbar_init(&x_full[b], 1);
+      mbar_init(&x_empty[b], 1);
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&t_full[b], 1);
-      mbar_init(&t_empty[b], 256);
+      mbar_init(&t_empty[b], 8);  // one epilogue group: 4 warps x 2 CTAs
+      mbar_init(&m_full[b], 4);
+      mbar_init(&m_empty[b], 4);
     }
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, 512);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_holder, 512);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // barriers and TMEM of both CTAs ready before any cross-CTA traffic
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const uint32_t x_base = smem_u32(smem + L::kX);
   const uint32_t st_base = smem_u32(smem + L::kStages);
 
   if (warp == 0 && lane == 0) {
-    // ---------------------------------------------------------- producer
-    prefetch_tmap(&tmap_x);
+    // ------------------------------------------ centroid producer (both)
     prefetch_tmap(&tmap_c);
     int st = 0;
     bool ok = true;
-    for (int pp = 0; pp < npairs && ok; ++pp) {
-      if (pp > 0 && !mbar_wait(x_empty, (pp - 1) & 1, abort_flag)) break;
-      const int row0 = bh * g.N + (pair0 + pp) * 256;
-      mbar_arrive_expect_tx(x_full, 2 * L::kXTileBytes);
-      for (int t = 0; t < 2; ++t)
-        for (int kb = 0; kb < L::kXBlocks; ++kb)
-          tma_load_2d(x_base + t * L::kXTileBytes + kb * 16384, &tmap_x, kb * 64, row0 + t * 128, x_full);
+    for (int i = 0; i < nunits && ok; ++i) {
+      const int bh = (int)((u0 + i) / uph);
       for (int c = 0; c < nchunks && ok; ++c) {
         for (int kb = 0; kb < kblocks; ++kb, ++st) {
           const int s = st % kAssignStages;
-          if (st >= kAssignStages && !mbar_wait(&c_empty[s], ((st / kAssignStages) - 1) & 1, abort_flag)) {
+          if (st >= kAssignStages && !mbar_wait_sleep(&c_empty[s], ((st / kAssignStages) - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&c_full[s], g.chunk * 128);
-          tma_load_2d(st_base + s * L::kStageBytes, &tmap_c, kb * 64, bh * g.c_pad + c * g.chunk, &c_full[s]);
+          if (rank == 0) mbar_arrive_expect_tx(&c_full[s], 2 * half * 128);
+          tma_load_2d_pair(st_base + s * L::kStageBytes, &tmap_c, kb * 64,
+                           bh * g.c_pad + c * g.chunk + (int)rank * half, mapa_shared(smem_u32(&c_full[s]), 0));
         }
       }
     }
-  } else if (warp == 1 && lane == 0) {
-    // -------------------------------------------------------------- MMA
-    const uint32_t idesc = umma_idesc_bf16(128, g.chunk, false, false);
+  } else if (warp == 2 && lane == 0) {
+    // --------------------------------------------- token producer (both)
+    prefetch_tmap(&tmap_x);
+    for (int i = 0; i < nunits; ++i) {
+      const int buf = i % kAssignXBufs;
+      if (i >= kAssignXBufs && !mbar_wait_sleep(&x_empty[buf], ((i / kAssignXBufs) - 1) & 1, abort_flag)) break;
+      const long long q = u0 + i;
+      const int bh = (int)(q / uph), pr = (int)(q % uph);
+      const int row = bh * g.N + pr * 256 + (int)rank * 128;
+      if (rank == 0) mbar_arrive_expect_tx(&x_full[buf], 2 * L::kXTileBytes);
+      const uint32_t bar = mapa_shared(smem_u32(&x_full[buf]), 0);
+      for (int kb = 0; kb < L::kXBlocks; ++kb)
+        tma_load_2d_pair(x_base + buf * L::kXTileBytes + kb * 16384, &tmap_x, kb * 64, row, bar);
+    }
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ------------------------------------------------------- MMA (leader)
+    const uint32_t idesc = umma_idesc_bf16(256, g.chunk, false, false);
     int st = 0, gc = 0;  // stage counter, global chunk counter (TMEM buffer phases)
     bool ok = true;
-    for (int pp = 0; pp < npairs && ok; ++pp) {
-      if (!mbar_wait(x_full, pp & 1, abort_flag)) break;
+    for (int i = 0; i < nunits && ok; ++i) {
+      const int buf = i % kAssignXBufs;
+      if (!mbar_wait_sleep(&x_full[buf], (i / kAssignXBufs) & 1, abort_flag)) break;
+      const uint32_t xb = x_base + buf * L::kXTileBytes;
       for (int c = 0; c < nchunks && ok; ++c, ++gc) {
         const int b = gc & 1;
-        if (gc >= 2 && !mbar_wait(&t_empty[b], ((gc >> 1) - 1) & 1, abort_flag)) {
+        if (gc >= 2 && !mbar_wait_sleep(&t_empty[b], ((gc >> 1) - 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         for (int kb = 0; kb < kblocks; ++kb, ++st) {
           const int s = st % kAssignStages;
-          if (!mbar_wait(&c_full[s], (st / kAssignStages) & 1, abort_flag)) {
+          if (!mbar_wait_sleep(&c_full[s], (st / kAssignStages) & 1, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const int xkb = kb % L::kXBlocks;
-          for (int t = 0; t < 2; ++t) {
-            const uint32_t dcol = tmem + (uint32_t)((b * 2 + t) * 128);
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t adesc =
-                  umma_desc_sw128(x_base + t * L::kXTileBytes + xkb * 16384 + k * 32, 16, 1024);
-              const uint64_t bdesc = umma_desc_sw128(st_base + s * L::kStageBytes + k * 32, 16, 1024);
-              umma_bf16_ss(dcol, adesc, bdesc, idesc, (kb | k) != 0);
-            }
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t adesc = umma_desc_sw128(xb + xkb * 16384 + k * 32, 16, 1024);
+            const uint64_t bdesc = umma_desc_sw128(st_base + s * L::kStageBytes + k * 32, 16, 1024);
+            umma_bf16_ss_pair(tmem + (uint32_t)(b * 256), adesc, bdesc, idesc, (kb | k) != 0);
           }
-          umma_commit(&c_empty[s]);
+          umma_commit_pair_mc(&c_empty[s], 3);
         }
         if (!ok) break;
-        umma_commit(&t_full[b]);
+        umma_commit_pair_mc(&t_full[b], 3);
       }
-      if (ok) umma_commit(x_empty);
+      if (ok) umma_commit_pair_mc(&x_empty[buf], 3);
     }
     // drain: every issued MMA completes before TMEM is released
-    umma_commit(fin);
+    umma_commit_pair(fin);
     mbar_wait_drain(fin, 0);
   } else if (warp >= 4) {
-    // --------------------------------------------------------- epilogue
-    const int t = (warp - 4) >> 2;          // tile 0 or 1
-    const int r = tid - 128 - t * 128;      // row inside the tile = TMEM lane
+    // ------------------------------------------------- epilogue (both)
+    const int grp = (warp - 4) >> 2;  // TMEM buffer this group reduces
+    const int r = (warp & 3) * 32 + lane;  // row of this CTA's tile = TMEM lane
     const uint32_t lane_off = (uint32_t)((r & ~31) << 16);
+    const uint32_t t_empty_lead = mapa_shared(smem_u32(&t_empty[grp]), 0);
     int gc = 0;
     bool ok = true;
-    for (int pp = 0; pp < npairs && ok; ++pp) {
+    for (int i = 0; i < nunits && ok; ++i) {
+      const long long q = u0 + i;
+      const int bh = (int)(q / uph), pr = (int)(q % uph);
+      const float* nrm = norms + (size_t)bh * g.c_pad;
       float best = __int_as_float(0x7f800000);
       int best_j = 0;
       for (int c = 0; c < nchunks; ++c, ++gc) {
         const int b = gc & 1;
-        if (!mbar_wait_warp(&t_full[b], (gc >> 1) & 1, abort_flag)) {
+        if (b != grp) continue;
+        // ||c||^2 of the chunk, fetched before the wait and kept in this
+        // warp's shared-memory slice; padding centroids have an infinite norm
+        // and columns past the chunk get one, so neither can win (an
+        // infinite distance never compares below `best`)
+        const float kInf = __int_as_float(0x7f800000);
+        const float4* nsrc = reinterpret_cast<const float4*>(nrm + c * g.chunk);
+        const float4 nl0 = (4 * lane < g.chunk) ? __ldg(nsrc + lane) : make_float4(kInf, kInf, kInf, kInf);
+        const float4 nl1 =
+            (4 * (lane + 32) < g.chunk) ? __ldg(nsrc + lane + 32) : make_float4(kInf, kInf, kInf, kInf);
+        if (!mbar_wait_warp_sleep(&t_full[b], (gc >> 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t col0 = tmem + lane_off + (uint32_t)((b * 2 + t) * 128);
-        for (int cb = 0; cb < g.chunk; cb += 32) {
-          float v[32];
-          tmem_ld32(col0 + cb, v);
+        __syncwarp();  // every lane is done with the previous chunk's norms
+        float4* nw = norms_s + (warp - 4) * 64;
+        nw[lane] = nl0;
+        nw[lane + 32] = nl1;
+        __syncwarp();
+        const uint32_t col0 = tmem + lane_off + (uint32_t)(b * 256);
+        // 32-column groups, the next group's TMEM load in flight while one is
+        // reduced (each wait covers the one load then outstanding)
+        float va[32], vb[32];
+        tmem_ld32(col0, va);
+        for (int cb = 0; cb < g.chunk; cb += 64) {
           tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int j = c * g.chunk + cb + e;
-            if (cb + e < g.chunk && j < g.C) {
-              const float dist = fmaf(-2.f, v[e], norm_s[j]);
-              if (dist < best) {
-                best = dist;
-                best_j = j;
-              }
-            }
+          pin_regs32(va);
+          if (cb + 32 < g.chunk) tmem_ld32(col0 + cb + 32, vb);
+          assign_reduce32(va, nw + cb / 4, cb, g.chunk, c * g.chunk + cb, best, best_j);
+          if (cb + 32 < g.chunk) {
+            tmem_wait_ld();
+            pin_regs32(vb);
+            if (cb + 64 < g.chunk) tmem_ld32(col0 + cb + 64, va);
+            assign_reduce32(vb, nw + cb / 4 + 8, cb + 32, g.chunk, c * g.chunk + cb + 32, best, best_j);
           }
         }
         tc_fence_before();
-        mbar_arrive(&t_empty[b]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(t_empty_lead);
       }
       if (!ok) break;
-      const int tok = (pair0 + pp) * 256 + t * 128 + r;
-      if (tok < g.N) assign[(size_t)bh * g.N + tok] = best_j;
+      // merge the two groups' minima of this unit (slot i & 1); on equal
+      // distances the lower centroid index wins
+      float2* slot = merge + (i & 1) * 128 + r;
+      if (grp == 1) {
+        if (i >= 2 && !mbar_wait_warp_sleep(&m_empty[i & 1], ((i >> 1) - 1) & 1, abort_flag)) break;
+        *slot = make_float2(best, __int_as_float(best_j));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&m_full[i & 1]);
+      } else {
+        if (!mbar_wait_warp_sleep(&m_full[i & 1], (i >> 1) & 1, abort_flag)) break;
+        const float2 o = *slot;
+        const int oj = __float_as_int(o.y);
+        const int jj = (o.x < best || (o.x == best && oj < best_j)) ? oj : best_j;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&m_empty[i & 1]);
+        const int tok = pr * 256 + (int)rank * 128 + r;
+        if (tok < g.N) assign[(size_t)bh * g.N + tok] = jj;
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // the peer is done with this CTA's barriers and TMEM
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
 cudaError_t launch_kmeans_assign(const KmeansGeom& g, const CUtensorMap* tmap_x, const CUtensorMap* tmap_c,
                                  const float* norms, int32_t* assign, cudaStream_t s) {
-  const int pairs = (g.N + 255) / 256;
-  dim3 grid((pairs + kPairsPerCta - 1) / kPairsPerCta, g.BH);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long units = (long long)g.BH * ((g.N + 255) / 256);
+  int npairs = sms / 2;
+  if (units < npairs) npairs = (int)units;
+  if (npairs < 1) npairs = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * npairs);
+  cfg.blockDim = dim3(kAssignThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (g.d == 128) {
-    const size_t sm = AssignSmem<128>::bytes(g.c_pad);
+    cfg.dynamicSmemBytes = AssignSmem<128>::bytes();
     cudaError_t e = cudaFuncSetAttribute(kmeans_assign_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sm);
+                                         (int)cfg.dynamicSmemBytes);
     if (e != cudaSuccess) return e;
-    kmeans_assign_kernel<128><<<grid, kAssignThreads, sm, s>>>(*tmap_x, *tmap_c, g, norms, assign);
-  } else {
-    const size_t sm = AssignSmem<64>::bytes(g.c_pad);
-    cudaError_t e = cudaFuncSetAttribute(kmeans_assign_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sm);
-    if (e != cudaSuccess) return e;
-    kmeans_assign_kernel<64><<<grid, kAssignThreads, sm, s>>>(*tmap_x, *tmap_c, g, norms, assign);
+    return cudaLaunchKernelEx(&cfg, kmeans_assign_kernel<128>, *tmap_x, *tmap_c, g, norms, assign);
   }
-  return cudaGetLastError();
+  cfg.dynamicSmemBytes = AssignSmem<64>::bytes();
+  cudaError_t e = cudaFuncSetAttribute(kmeans_assign_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)cfg.dynamicSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, kmeans_assign_kernel<64>, *tmap_x, *tmap_c, g, norms, assign);
 }
 
 // ------------------------------------------------------------------ update
@@ -358,6 +478,7 @@ __global__ void __launch_bounds__(kUpdThreads)
                          __nv_bfloat16* __restrict__ cmma, float* __restrict__ norms, float* __restrict__ partial,
                          int32_t* __restrict__ arrive, int part_slots) {
   __shared__ float part[kUpdThreads * 8];
+  __shared__ int rows_s[kUpdRows];  // the piece's token indices
   __shared__ float red[32];
   __shared__ int scan_np[kUpdThreads / 32], scan_mp[kUpdThreads / 32];
   __shared__ int s_c, s_piece, s_np, s_base, s_last;
@@ -424,6 +545,8 @@ __global__ void __launch_bounds__(kUpdThreads)
   const int lo = off[c], hi = off[c + 1];
   const int plo = lo + piece * kUpdRows, phi = min(hi, plo + kUpdRows);
   const int32_t* prow = perm + (size_t)bh * g.N;
+  for (int p = plo + tid; p < phi; p += kUpdThreads) rows_s[p - plo] = prow[p];
+  __syncthreads();
   const __nv_bfloat16* xh = X + (size_t)bh * g.N * g.d + ch * 8;
   float acc[8];
 #pragma unroll
@@ -434,7 +557,7 @@ __global__ void __launch_bounds__(kUpdThreads)
 #pragma unroll
     for (int u = 0; u < kUpdUnroll; ++u) {
       const int p = p0 + u * slots;
-      src[u] = p < phi ? prow[p] : -1;
+      src[u] = p < phi ? rows_s[p - plo] : -1;
     }
 #pragma unroll
     for (int u = 0; u < kUpdUnroll; ++u) {
