@@ -230,18 +230,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
     // issued lane -> 16-byte chunk of a row, so one warp instruction moves
     // whole 256-byte rows (full L2 sectors).
     const int pw = tp >> 5;
-    auto key_pos = [&](int j, int r) -> int {  // -1: padding slot
-      const int l = j * 128 + r;               // slot of tile row r in the key list
+    // Slot -> permuted key position.  Each row stream of a lane visits
+    // increasing slots (one per tile), so its exact group e (the last with
+    // gpre[e] <= slot) is found by walking forward from the previous one,
+    // about one step per tile, instead of a binary search per slot.
+    auto key_pos = [&](int j, int r, int& e) -> int {  // -1: padding slot
+      const int l = j * 128 + r;                       // slot of tile row r in the key list
       if (l < Xi) {
-        int lo = 0, hi = n_exact - 1;  // last e with gpre[e] <= l
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (gpre[mid] <= l)
-            lo = mid;
-          else
-            hi = mid - 1;
-        }
-        return gstart[lo] + (l - gpre[lo]);
+        while (e + 1 < n_exact && gpre[e + 1] <= l) ++e;
+        return gstart[e] + (l - gpre[e]);
       }
       if (l < Lk) return __ldg(spos + (l - Xi));
       return -1;
@@ -271,13 +268,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
                     p < 0 ? 0u : 16u);
       }
     };
-    int nA = key_pos(0, 64 * pw + lane), nB = key_pos(0, 64 * pw + 32 + lane);
+    int eA = 0, eB = 0;  // exact-group cursors of the two row streams
+    int nA = key_pos(0, 64 * pw + lane, eA), nB = key_pos(0, 64 * pw + 32 + lane, eB);
     for (int kt = 0; kt < ntk; ++kt) {
       const int s = kt & 1, use = kt >> 1;
       const int posA = checked(nA), posB = checked(nB);
       if (kt + 1 < ntk) {
-        nA = key_pos(kt + 1, 64 * pw + lane);
-        nB = key_pos(kt + 1, 64 * pw + 32 + lane);
+        nA = key_pos(kt + 1, 64 * pw + lane, eA);
+        nB = key_pos(kt + 1, 64 * pw + 32 + lane, eB);
       }
       if (kt >= 2 && !mbar_wait(&k_empty[s], (use - 1) & 1, abort_flag)) break;
       issue_rows(a.Kp, k_s + s * L::kTileBytes, posA, posB);
