@@ -9,7 +9,7 @@ binding raises.
 
 Entry points (same names as the C ABI, without the ``instagen_`` prefix):
 ``cluster``, ``permutation``, ``gather``, ``select_sample``, ``attention``,
-``forward`` plus ``make_params``, ``exact_budget``, ``sample_budget``,
+``forward``, ``forward_host`` plus ``make_params``, ``exact_budget``, ``sample_budget``,
 ``workspace_size``, ``forward_layout`` and ``device_status``.
 """
 from __future__ import annotations
@@ -52,7 +52,7 @@ _SYMBOLS = ("instagen_exact_budget", "instagen_sample_budget", "instagen_workspa
             "instagen_cluster_workspace_size", "instagen_error_string", "instagen_device_status",
             "instagen_cluster", "instagen_permutation", "instagen_gather", "instagen_select_sample",
             "instagen_attention", "instagen_forward", "instagen_forward_layout_get",
-            "instagen_cluster_static")
+            "instagen_cluster_static", "instagen_forward_host_workspace_size", "instagen_forward_host")
 
 
 def lib():
@@ -80,6 +80,8 @@ def lib():
         "instagen_forward": (ctypes.c_int, [PP, PP, PP, PP, P, PP, sz, vp]),
         "instagen_forward_layout_get": (ctypes.c_int, [P, ctypes.POINTER(ForwardLayout)]),
         "instagen_cluster_static": (ctypes.c_int, [PP, i32, i32, PP, P, PP, PP, PP, PP, vp]),
+        "instagen_forward_host_workspace_size": (sz, [P, i32]),
+        "instagen_forward_host": (ctypes.c_int, [PP, PP, PP, PP, P, i32, PP, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -273,6 +275,36 @@ def forward(Q, K, V, p: Params, workspace: Optional[torch.Tensor] = None,
     _need(O, "O", torch.bfloat16, _bhnd(p))
     _check(lib().instagen_forward(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), ctypes.byref(p), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream()), "instagen_forward")
+    return O
+
+
+def forward_host_workspace_size(p: Params, heads_per_chunk: int = 0) -> int:
+    return int(lib().instagen_forward_host_workspace_size(ctypes.byref(p), heads_per_chunk))
+
+
+def forward_host(Q, K, V, p: Params, out: Optional[torch.Tensor] = None, heads_per_chunk: int = 0,
+                 workspace: Optional[torch.Tensor] = None, device=None) -> torch.Tensor:
+    """The whole call on HOST tensors (CPU, contiguous bf16 [B,H,N,d];
+    page-locked for overlapped copies): head chunks are copied in, computed
+    and copied out in a pipeline on the current CUDA stream.  Returns the host
+    output O (synchronise the stream before reading it)."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        if not isinstance(t, torch.Tensor) or t.is_cuda:
+            raise InstaGenError(f"{n} must be a host (CPU) tensor")
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or tuple(t.shape) != _bhnd(p):
+            raise ValueError(f"{n} must be contiguous bf16 {_bhnd(p)}")
+    O = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=Q.is_pinned()) if out is None else out
+    if O.is_cuda or O.dtype != torch.bfloat16 or not O.is_contiguous() or tuple(O.shape) != _bhnd(p):
+        raise ValueError(f"out must be a contiguous host bf16 tensor {_bhnd(p)}")
+    nws = forward_host_workspace_size(p, heads_per_chunk)
+    if nws == 0:
+        raise InstaGenError("invalid parameters for instagen_forward_host")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    ws = torch.empty(nws, dtype=torch.uint8, device=dev) if workspace is None else workspace
+    if ws.numel() * ws.element_size() < nws:
+        raise InstaGenError(f"workspace too small: {ws.numel() * ws.element_size()} < {nws}")
+    _check(lib().instagen_forward_host(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), ctypes.byref(p), heads_per_chunk,
+                                       _ptr(ws), ws.numel() * ws.element_size(), _stream()), "instagen_forward_host")
     return O
 
 

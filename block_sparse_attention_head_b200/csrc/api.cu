@@ -151,6 +151,112 @@ int forward_layout(const instagen_params* p, instagen_forward_layout* L) {
   return IG_OK;
 }
 
+// bh0: global index of the first head (the sample's Philox counter uses it).
+int select_impl(const float* cq, const float* ck, const int32_t* k_offsets, const instagen_params* p,
+                int32_t* exact_groups, int32_t* counts, int32_t* sample_pos, float* sample_bias, int bh0,
+                void* stream) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if ((rc = check_clusters(p->Cq)) || (rc = check_clusters(p->Ck))) return rc;
+  if ((rc = check_budgets(p))) return rc;
+  const long long m = budget(p->sample_frac, p->N);
+  if (!cq || !ck || !k_offsets || !exact_groups || !counts) return IG_ERR_INVALID_ARG;
+  if (m > 0 && (!sample_pos || !sample_bias)) return IG_ERR_INVALID_ARG;
+  ig::SelectArgs a;
+  a.cq = cq;
+  a.ck = ck;
+  a.k_offsets = k_offsets;
+  a.BH = p->B * p->H;
+  a.Cq = p->Cq;
+  a.Ck = p->Ck;
+  a.d = p->d;
+  a.scale = p->softmax_scale;
+  a.E = budget(p->exact_frac, p->N);
+  a.m = m;
+  a.seed = p->seed;
+  a.layer = p->layer;
+  a.mode = p->sampling;
+  a.bh0 = bh0;
+  a.exact_groups = exact_groups;
+  a.counts = counts;
+  a.sample_pos = sample_pos;
+  a.sample_bias = sample_bias;
+  return cuda_status(ig::launch_select_sample(a, static_cast<cudaStream_t>(stream)));
+}
+
+
+// The whole call on device buffers; bh0 = global index of the first head.
+int forward_impl(const void* Q, const void* K, const void* V, void* O, const instagen_params* p, void* ws,
+                 size_t ws_bytes, int bh0, void* stream) {
+  instagen_forward_layout L;
+  int rc = forward_layout(p, &L);
+  if (rc) return rc;
+  if (p->Ck > ig::kAttnMaxExactGroups) return IG_ERR_UNSUPPORTED;
+  if (p->kmeans_iters < 1 || p->kmeans_iters > 10000) return IG_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return IG_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return IG_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  float* cq = reinterpret_cast<float*>(w + L.cq);
+  float* ck = reinterpret_cast<float*>(w + L.ck);
+  int32_t* qa = reinterpret_cast<int32_t*>(w + L.q_assign);
+  int32_t* ka = reinterpret_cast<int32_t*>(w + L.k_assign);
+  int32_t* qp = reinterpret_cast<int32_t*>(w + L.q_perm);
+  int32_t* kp = reinterpret_cast<int32_t*>(w + L.k_perm);
+  int32_t* qo = reinterpret_cast<int32_t*>(w + L.q_offsets);
+  int32_t* ko = reinterpret_cast<int32_t*>(w + L.k_offsets);
+  void* Kp = w + L.kp;
+  void* Vp = w + L.vp;
+  int32_t* eg = reinterpret_cast<int32_t*>(w + L.exact_groups);
+  int32_t* cnt = reinterpret_cast<int32_t*>(w + L.counts);
+  int32_t* sp = reinterpret_cast<int32_t*>(w + L.sample_pos);
+  float* sb = reinterpret_cast<float*>(w + L.sample_bias);
+  void* cws = w + L.cluster_ws;
+  const size_t cws_bytes = L.total - L.cluster_ws;
+  rc = run_cluster(Q, p->Cq, p->kmeans_iters, nullptr, p, cq, qa, qp, qo, cws, cws_bytes, s);
+  if (rc) return rc;
+  rc = run_cluster(K, p->Ck, p->kmeans_iters, nullptr, p, ck, ka, kp, ko, cws, cws_bytes, s);
+  if (rc) return rc;
+  rc = cuda_status(ig::launch_gather_rows(static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V),
+                                          kp, p->B * p->H, p->N, p->d, Kp, Vp, false, true, s));
+  if (rc) return rc;
+  rc = select_impl(cq, ck, ko, p, eg, cnt, sp, sb, bh0, stream);
+  if (rc) return rc;
+  return instagen_attention(Q, Kp, Vp, qp, qo, ko, eg, cnt, sp, sb, p, O, stream);
+}
+
+
+// ------------------------------------------------------ host-buffer pipeline
+struct HostLayout {
+  int hc;                 // heads per chunk (at most)
+  size_t tensor;          // bytes of one chunk of one tensor (256-aligned)
+  size_t fwd_off, fwd;    // instagen_forward workspace of one chunk (two of them)
+  size_t total;
+};
+
+int host_layout(const instagen_params* p, int heads_per_chunk, HostLayout* L) {
+  const size_t head_bytes = (size_t)p->N * p->d * 2;
+  int hc = heads_per_chunk;
+  if (hc <= 0) {  // about 160 MB per tensor per chunk
+    const size_t k = ((size_t)160 << 20) / head_bytes;
+    hc = (int)(k < 1 ? 1 : (k > (size_t)p->H ? (size_t)p->H : k));
+  }
+  if (hc > p->H) hc = p->H;
+  instagen_params pc = *p;
+  pc.B = 1;
+  pc.H = hc;
+  instagen_forward_layout fl;
+  const int rc = forward_layout(&pc, &fl);
+  if (rc) return rc;
+  L->hc = hc;
+  L->tensor = align256((size_t)hc * head_bytes);
+  L->fwd_off = 8 * L->tensor;  // two slots x (Q, K, V, O)
+  L->fwd = fl.total;
+  L->total = L->fwd_off + 2 * align256(fl.total);
+  return IG_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -236,32 +342,7 @@ int instagen_gather(const void* X, const int32_t* perm, const instagen_params* p
 int instagen_select_sample(const float* cq, const float* ck, const int32_t* k_offsets, const instagen_params* p,
                            int32_t* exact_groups, int32_t* counts, int32_t* sample_pos, float* sample_bias,
                            void* stream) {
-  int rc = check_params(p);
-  if (rc) return rc;
-  if ((rc = check_clusters(p->Cq)) || (rc = check_clusters(p->Ck))) return rc;
-  if ((rc = check_budgets(p))) return rc;
-  const long long m = budget(p->sample_frac, p->N);
-  if (!cq || !ck || !k_offsets || !exact_groups || !counts) return IG_ERR_INVALID_ARG;
-  if (m > 0 && (!sample_pos || !sample_bias)) return IG_ERR_INVALID_ARG;
-  ig::SelectArgs a;
-  a.cq = cq;
-  a.ck = ck;
-  a.k_offsets = k_offsets;
-  a.BH = p->B * p->H;
-  a.Cq = p->Cq;
-  a.Ck = p->Ck;
-  a.d = p->d;
-  a.scale = p->softmax_scale;
-  a.E = budget(p->exact_frac, p->N);
-  a.m = m;
-  a.seed = p->seed;
-  a.layer = p->layer;
-  a.mode = p->sampling;
-  a.exact_groups = exact_groups;
-  a.counts = counts;
-  a.sample_pos = sample_pos;
-  a.sample_bias = sample_bias;
-  return cuda_status(ig::launch_select_sample(a, static_cast<cudaStream_t>(stream)));
+  return select_impl(cq, ck, k_offsets, p, exact_groups, counts, sample_pos, sample_bias, 0, stream);
 }
 
 int instagen_attention(const void* Q, const void* Kp, const void* Vp, const int32_t* q_perm,
@@ -302,42 +383,107 @@ int instagen_attention(const void* Q, const void* Kp, const void* Vp, const int3
 
 int instagen_forward(const void* Q, const void* K, const void* V, void* O, const instagen_params* p, void* ws,
                      size_t ws_bytes, void* stream) {
-  instagen_forward_layout L;
-  int rc = forward_layout(p, &L);
-  if (rc) return rc;
-  if (p->Ck > ig::kAttnMaxExactGroups) return IG_ERR_UNSUPPORTED;
-  if (p->kmeans_iters < 1 || p->kmeans_iters > 10000) return IG_ERR_INVALID_ARG;
-  if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
-    return IG_ERR_INVALID_ARG;
-  if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return IG_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  char* w = static_cast<char*>(ws);
-  float* cq = reinterpret_cast<float*>(w + L.cq);
-  float* ck = reinterpret_cast<float*>(w + L.ck);
-  int32_t* qa = reinterpret_cast<int32_t*>(w + L.q_assign);
-  int32_t* ka = reinterpret_cast<int32_t*>(w + L.k_assign);
-  int32_t* qp = reinterpret_cast<int32_t*>(w + L.q_perm);
-  int32_t* kp = reinterpret_cast<int32_t*>(w + L.k_perm);
-  int32_t* qo = reinterpret_cast<int32_t*>(w + L.q_offsets);
-  int32_t* ko = reinterpret_cast<int32_t*>(w + L.k_offsets);
-  void* Kp = w + L.kp;
-  void* Vp = w + L.vp;
-  int32_t* eg = reinterpret_cast<int32_t*>(w + L.exact_groups);
-  int32_t* cnt = reinterpret_cast<int32_t*>(w + L.counts);
-  int32_t* sp = reinterpret_cast<int32_t*>(w + L.sample_pos);
-  float* sb = reinterpret_cast<float*>(w + L.sample_bias);
-  void* cws = w + L.cluster_ws;
-  const size_t cws_bytes = L.total - L.cluster_ws;
-  rc = run_cluster(Q, p->Cq, p->kmeans_iters, nullptr, p, cq, qa, qp, qo, cws, cws_bytes, s);
-  if (rc) return rc;
-  rc = run_cluster(K, p->Ck, p->kmeans_iters, nullptr, p, ck, ka, kp, ko, cws, cws_bytes, s);
-  if (rc) return rc;
-  rc = cuda_status(ig::launch_gather_rows(static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V),
-                                          kp, p->B * p->H, p->N, p->d, Kp, Vp, false, true, s));
-  if (rc) return rc;
-  rc = instagen_select_sample(cq, ck, ko, p, eg, cnt, sp, sb, stream);
-  if (rc) return rc;
-  return instagen_attention(Q, Kp, Vp, qp, qo, ko, eg, cnt, sp, sb, p, O, stream);
+  return forward_impl(Q, K, V, O, p, ws, ws_bytes, 0, stream);
 }
 
+size_t instagen_forward_host_workspace_size(const instagen_params* p, int32_t heads_per_chunk) {
+  HostLayout L;
+  if (check_params(p) || heads_per_chunk < 0 || host_layout(p, heads_per_chunk, &L)) return 0;
+  return L.total;
+}
+
+int instagen_forward_host(const void* Q, const void* K, const void* V, void* O, const instagen_params* p,
+                          int32_t heads_per_chunk, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if (heads_per_chunk < 0 || !Q || !K || !V || !O) return IG_ERR_INVALID_ARG;
+  HostLayout L;
+  if ((rc = host_layout(p, heads_per_chunk, &L))) return rc;
+  if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return IG_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t s_in = nullptr, s_out = nullptr, s_c1 = nullptr;
+  cudaEvent_t ev[10] = {};  // start, in[2], comp[2], out[2], in done, out done, compute-1 done
+  bool ok = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&s_c1, cudaStreamNonBlocking) == cudaSuccess;
+  for (int i = 0; i < 10 && ok; ++i) ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+  cudaEvent_t ev_start = ev[0], *ev_in = ev + 1, *ev_comp = ev + 3, *ev_out = ev + 5;
+  cudaEvent_t ev_in_done = ev[7], ev_out_done = ev[8], ev_c1_done = ev[9];
+  // chunks alternate between two compute streams (the caller's and one of
+  // ours), each with its own forward workspace, so one chunk's tail overlaps
+  // the next chunk's first kernels
+  rc = ok ? IG_OK : IG_ERR_CUDA;
+  char* w = static_cast<char*>(ws);
+  const size_t head_bytes = (size_t)p->N * p->d * 2;
+  const char* hq = static_cast<const char*>(Q);
+  const char* hk = static_cast<const char*>(K);
+  const char* hv = static_cast<const char*>(V);
+  char* ho = static_cast<char*>(O);
+  if (rc == IG_OK) {
+    ok = cudaEventRecord(ev_start, s) == cudaSuccess && cudaStreamWaitEvent(s_in, ev_start, 0) == cudaSuccess &&
+         cudaStreamWaitEvent(s_out, ev_start, 0) == cudaSuccess &&
+         cudaStreamWaitEvent(s_c1, ev_start, 0) == cudaSuccess;
+    if (!ok) rc = IG_ERR_CUDA;
+  }
+  // chunk sizes of a batch row: a small first chunk (short pipeline fill),
+  // then hc heads, and a small last chunk (short drain)
+  const int q = L.hc / 4 > 1 ? L.hc / 4 : 1;
+  auto chunk_at = [&](int h) {
+    const int left = p->H - h;
+    if (h == 0) return left < q ? left : q;
+    if (left <= q) return left;
+    if (left <= L.hc + q) return left - q;
+    return L.hc;
+  };
+  int c = 0;
+  for (int b = 0; b < p->B && rc == IG_OK; ++b) {
+    for (int h0 = 0, n = 0; h0 < p->H && rc == IG_OK; h0 += n, ++c) {
+      n = chunk_at(h0);
+      const int slot = c & 1;
+      const size_t off = ((size_t)b * p->H + h0) * head_bytes, bytes = (size_t)n * head_bytes;
+      char* dq = w + (4 * slot + 0) * L.tensor;
+      char* dk = w + (4 * slot + 1) * L.tensor;
+      char* dv = w + (4 * slot + 2) * L.tensor;
+      char* dout = w + (4 * slot + 3) * L.tensor;
+      // copy in: the slot's inputs are free once chunk c - 2 is computed
+      ok = (c < 2 || cudaStreamWaitEvent(s_in, ev_comp[slot], 0) == cudaSuccess) &&
+           cudaMemcpyAsync(dq, hq + off, bytes, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+           cudaMemcpyAsync(dk, hk + off, bytes, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+           cudaMemcpyAsync(dv, hv + off, bytes, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+           cudaEventRecord(ev_in[slot], s_in) == cudaSuccess;
+      // compute (stream of this slot): after the copy in, and once chunk
+      // c - 2's output left the slot
+      cudaStream_t cs = slot ? s_c1 : s;
+      ok = ok && cudaStreamWaitEvent(cs, ev_in[slot], 0) == cudaSuccess &&
+           (c < 2 || cudaStreamWaitEvent(cs, ev_out[slot], 0) == cudaSuccess);
+      if (!ok) {
+        rc = IG_ERR_CUDA;
+        break;
+      }
+      instagen_params pc = *p;
+      pc.B = 1;
+      pc.H = n;
+      rc = forward_impl(dq, dk, dv, dout, &pc, w + L.fwd_off + slot * align256(L.fwd), L.fwd, b * p->H + h0, cs);
+      if (rc) break;
+      // copy out
+      ok = cudaEventRecord(ev_comp[slot], cs) == cudaSuccess &&
+           cudaStreamWaitEvent(s_out, ev_comp[slot], 0) == cudaSuccess &&
+           cudaMemcpyAsync(ho + off, dout, bytes, cudaMemcpyDeviceToHost, s_out) == cudaSuccess &&
+           cudaEventRecord(ev_out[slot], s_out) == cudaSuccess;
+      if (!ok) rc = IG_ERR_CUDA;
+    }
+  }
+  // `stream` is ordered after everything enqueued on the copy streams, also
+  // on an error (so synchronising it covers every pending host access)
+  if (s_in && ev_in_done && cudaEventRecord(ev_in_done, s_in) == cudaSuccess) cudaStreamWaitEvent(s, ev_in_done, 0);
+  if (s_out && ev_out_done && cudaEventRecord(ev_out_done, s_out) == cudaSuccess)
+    cudaStreamWaitEvent(s, ev_out_done, 0);
+  if (s_c1 && ev_c1_done && cudaEventRecord(ev_c1_done, s_c1) == cudaSuccess) cudaStreamWaitEvent(s, ev_c1_done, 0);
+  for (int i = 0; i < 10; ++i)
+    if (ev[i]) cudaEventDestroy(ev[i]);  // released once their work completes
+  if (s_in) cudaStreamDestroy(s_in);
+  if (s_out) cudaStreamDestroy(s_out);
+  if (s_c1) cudaStreamDestroy(s_c1);
+  return rc;
+}
 }  // extern "C"

@@ -60,6 +60,7 @@ struct SelectArgs {
   unsigned long long seed;
   unsigned layer;
   int mode;
+  int bh0;  // global index of head 0 of this launch (the Philox counter's head)
   int32_t* exact_groups;
   int32_t* counts;
   int32_t* sample_pos;

@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(kSelThreads)
     int32_t pos = -1;
     float bias = 0.0f;
     if (t < draws) {
-      const U4 rnd = philox4x32_10(U4{(uint32_t)t, (uint32_t)i, (uint32_t)bh, a.layer}, k0, k1);
+      const U4 rnd = philox4x32_10(U4{(uint32_t)t, (uint32_t)i, (uint32_t)(a.bh0 + bh), a.layer}, k0, k1);
       const unsigned long long u = ((unsigned long long)rnd.y << 32) | rnd.x;
       const unsigned long long r = __umul64hi(u, T);
       int lo = 0, hi = Ck - 1;  // first j with cdf[j] > r

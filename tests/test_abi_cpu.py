@@ -88,6 +88,23 @@ def test_null_pointers_and_workspace_rejected(lib):
                                   ctypes.byref(big), fake, None) == 2             # Ck > 2048
 
 
+def test_forward_host_checks_on_host(lib):
+    p = ig.make_params(2, 5, 1000, 128, 8, 16)
+    L1 = lib.instagen_workspace_size(ctypes.byref(ig.make_params(1, 2, 1000, 128, 8, 16)))
+    # two staging slots of 2 heads x (Q, K, V, O) plus one chunk's forward workspace
+    assert lib.instagen_forward_host_workspace_size(ctypes.byref(p), 2) >= 8 * 2 * 1000 * 128 * 2 + L1
+    assert lib.instagen_forward_host_workspace_size(ctypes.byref(p), -1) == 0
+    # automatic chunk: all 5 small heads in one chunk
+    L5 = lib.instagen_workspace_size(ctypes.byref(ig.make_params(1, 5, 1000, 128, 8, 16)))
+    assert lib.instagen_forward_host_workspace_size(ctypes.byref(p), 0) >= L5
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: rejected before any copy or launch
+    assert lib.instagen_forward_host(None, fake, fake, fake, ctypes.byref(p), 2, fake, 1 << 30, None) == 1
+    assert lib.instagen_forward_host(fake, fake, fake, fake, ctypes.byref(p), -3, fake, 1 << 30, None) == 1
+    assert lib.instagen_forward_host(fake, fake, fake, fake, ctypes.byref(p), 2, fake, 16, None) == 3
+    bad = ig.make_params(1, 2, 1000, 96, 8, 16)
+    assert lib.instagen_forward_host(fake, fake, fake, fake, ctypes.byref(bad), 1, fake, 1 << 30, None) == 2
+
+
 def test_error_strings(lib):
     for code in range(6):
         assert lib.instagen_error_string(code)
