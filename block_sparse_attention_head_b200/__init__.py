@@ -52,7 +52,8 @@ _SYMBOLS = ("instagen_exact_budget", "instagen_sample_budget", "instagen_workspa
             "instagen_cluster_workspace_size", "instagen_error_string", "instagen_device_status",
             "instagen_cluster", "instagen_permutation", "instagen_gather", "instagen_select_sample",
             "instagen_attention", "instagen_forward", "instagen_forward_layout_get",
-            "instagen_cluster_static", "instagen_forward_host_workspace_size", "instagen_forward_host")
+            "instagen_cluster_static", "instagen_forward_host_workspace_size", "instagen_forward_host",
+            "instagen_forward_init")
 
 
 def lib():
@@ -82,6 +83,7 @@ def lib():
         "instagen_cluster_static": (ctypes.c_int, [PP, i32, i32, PP, P, PP, PP, PP, PP, vp]),
         "instagen_forward_host_workspace_size": (sz, [P, i32]),
         "instagen_forward_host": (ctypes.c_int, [PP, PP, PP, PP, P, i32, PP, sz, vp]),
+        "instagen_forward_init": (ctypes.c_int, [PP, PP, PP, PP, P, PP, PP, PP, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -263,8 +265,11 @@ def attention(Q, Kp, Vp, q_perm, q_offsets, k_offsets, exact_groups, counts, sam
 
 
 def forward(Q, K, V, p: Params, workspace: Optional[torch.Tensor] = None,
-            out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """The whole InstaGen attention call; O [B,H,N,d] bf16 in original order."""
+            out: Optional[torch.Tensor] = None, cq_init: Optional[torch.Tensor] = None,
+            ck_init: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The whole InstaGen attention call; O [B,H,N,d] bf16 in original order.
+    cq_init / ck_init (fp32 [B,H,C,d] on the device): warm-start centroids
+    (instagen_forward_init), e.g. the previous call's ``forward_intermediates``."""
     for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
         _need(t, n, torch.bfloat16, _bhnd(p))
     nws = workspace_size(p)
@@ -273,8 +278,17 @@ def forward(Q, K, V, p: Params, workspace: Optional[torch.Tensor] = None,
         raise InstaGenError(f"workspace too small: {ws.numel() * ws.element_size()} < {nws}")
     O = torch.empty_like(Q) if out is None else out
     _need(O, "O", torch.bfloat16, _bhnd(p))
-    _check(lib().instagen_forward(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), ctypes.byref(p), _ptr(ws),
-                                  ws.numel() * ws.element_size(), _stream()), "instagen_forward")
+    if cq_init is None and ck_init is None:
+        _check(lib().instagen_forward(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), ctypes.byref(p), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream()), "instagen_forward")
+        return O
+    if cq_init is not None:
+        _need(cq_init, "cq_init", torch.float32, (p.B, p.H, p.Cq, p.d))
+    if ck_init is not None:
+        _need(ck_init, "ck_init", torch.float32, (p.B, p.H, p.Ck, p.d))
+    _check(lib().instagen_forward_init(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), ctypes.byref(p), _ptr(cq_init),
+                                       _ptr(ck_init), _ptr(ws), ws.numel() * ws.element_size(), _stream()),
+           "instagen_forward_init")
     return O
 
 

@@ -185,9 +185,10 @@ int select_impl(const float* cq, const float* ck, const int32_t* k_offsets, cons
 }
 
 
-// The whole call on device buffers; bh0 = global index of the first head.
-int forward_impl(const void* Q, const void* K, const void* V, void* O, const instagen_params* p, void* ws,
-                 size_t ws_bytes, int bh0, void* stream) {
+// The whole call on device buffers; bh0 = global index of the first head;
+// cq_init / ck_init: initial centroids or null (token floor(j*N/C)).
+int forward_impl(const void* Q, const void* K, const void* V, void* O, const instagen_params* p,
+                 const float* cq_init, const float* ck_init, void* ws, size_t ws_bytes, int bh0, void* stream) {
   instagen_forward_layout L;
   int rc = forward_layout(p, &L);
   if (rc) return rc;
@@ -214,9 +215,9 @@ int forward_impl(const void* Q, const void* K, const void* V, void* O, const ins
   float* sb = reinterpret_cast<float*>(w + L.sample_bias);
   void* cws = w + L.cluster_ws;
   const size_t cws_bytes = L.total - L.cluster_ws;
-  rc = run_cluster(Q, p->Cq, p->kmeans_iters, nullptr, p, cq, qa, qp, qo, cws, cws_bytes, s);
+  rc = run_cluster(Q, p->Cq, p->kmeans_iters, cq_init, p, cq, qa, qp, qo, cws, cws_bytes, s);
   if (rc) return rc;
-  rc = run_cluster(K, p->Ck, p->kmeans_iters, nullptr, p, ck, ka, kp, ko, cws, cws_bytes, s);
+  rc = run_cluster(K, p->Ck, p->kmeans_iters, ck_init, p, ck, ka, kp, ko, cws, cws_bytes, s);
   if (rc) return rc;
   rc = cuda_status(ig::launch_gather_rows(static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V),
                                           kp, p->B * p->H, p->N, p->d, Kp, Vp, false, true, s));
@@ -383,7 +384,12 @@ int instagen_attention(const void* Q, const void* Kp, const void* Vp, const int3
 
 int instagen_forward(const void* Q, const void* K, const void* V, void* O, const instagen_params* p, void* ws,
                      size_t ws_bytes, void* stream) {
-  return forward_impl(Q, K, V, O, p, ws, ws_bytes, 0, stream);
+  return forward_impl(Q, K, V, O, p, nullptr, nullptr, ws, ws_bytes, 0, stream);
+}
+
+int instagen_forward_init(const void* Q, const void* K, const void* V, void* O, const instagen_params* p,
+                          const float* cq_init, const float* ck_init, void* ws, size_t ws_bytes, void* stream) {
+  return forward_impl(Q, K, V, O, p, cq_init, ck_init, ws, ws_bytes, 0, stream);
 }
 
 size_t instagen_forward_host_workspace_size(const instagen_params* p, int32_t heads_per_chunk) {
@@ -463,7 +469,8 @@ int instagen_forward_host(const void* Q, const void* K, const void* V, void* O, 
       instagen_params pc = *p;
       pc.B = 1;
       pc.H = n;
-      rc = forward_impl(dq, dk, dv, dout, &pc, w + L.fwd_off + slot * align256(L.fwd), L.fwd, b * p->H + h0, cs);
+      rc = forward_impl(dq, dk, dv, dout, &pc, nullptr, nullptr, w + L.fwd_off + slot * align256(L.fwd), L.fwd,
+                        b * p->H + h0, cs);
       if (rc) break;
       // copy out
       ok = cudaEventRecord(ev_comp[slot], cs) == cudaSuccess &&

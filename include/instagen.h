@@ -220,6 +220,20 @@ int instagen_forward(const void* Q, const void* K, const void* V, void* O, const
                      size_t ws_bytes, void* stream);
 
 /*
+ * instagen_forward with initial centroids for both clusterings (a warm
+ * start, e.g. from the previous denoising step's centroids, run with fewer
+ * k-means iterations).  No separate counterpart on the pages; it serves the
+ * step-to-step reuse of the clustering that the pages' warm-up/step
+ * structure invites.  cq_init [B,H,Cq,d] and ck_init [B,H,Ck,d] fp32 device
+ * pointers, each may be NULL (that clustering starts from tokens
+ * floor(j*N/C)).  They may point at the cq / ck blocks of the same workspace
+ * (instagen_forward_layout: the previous call's final centroids): each row
+ * is read before it is overwritten.  Otherwise as instagen_forward.
+ */
+int instagen_forward_init(const void* Q, const void* K, const void* V, void* O, const instagen_params* p,
+                          const float* cq_init, const float* ck_init, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * instagen_forward with HOST buffers: Q, K, V (inputs) and O (output) are
  * host memory in the [B,H,N,d] bf16 layout of instagen_forward.  No
  * counterpart on the method's pages: the heads are independent, so the call

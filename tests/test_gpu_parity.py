@@ -324,6 +324,33 @@ def test_forward_error_vs_dense_tracks_oracle(oracle_runs):
     ig.device_status()
 
 
+def test_forward_warm_start():
+    """instagen_forward_init: k-means starts from given centroids (here the
+    previous call's, read from its workspace).  Its intermediates equal the
+    staged instagen_cluster calls with the same init, and passing the
+    workspace's own centroid blocks as the init (aliased) gives the same
+    output as a separate copy of them."""
+    p, Q, K, V = _inputs("ragged_d128")
+    Q, K, V = Q.cuda(), K.cuda(), V.cuda()
+    ws0 = torch.empty(ig.workspace_size(p), dtype=torch.uint8, device="cuda")
+    ig.forward(Q, K, V, p, workspace=ws0)
+    it0 = ig.forward_intermediates(ws0, p)
+    cq0, ck0 = it0["cq"].clone(), it0["ck"].clone()
+    p2 = ig.make_params(p.B, p.H, p.N, p.d, p.Cq, p.Ck, iters=2, exact_frac=p.exact_frac,
+                        sample_frac=p.sample_frac, seed=p.seed, layer=p.layer, sampling=p.sampling)
+    ws1 = torch.empty_like(ws0)
+    O1 = ig.forward(Q, K, V, p2, workspace=ws1, cq_init=cq0, ck_init=ck0)
+    it1 = ig.forward_intermediates(ws1, p2)
+    for X, C, init, names in ((Q, p.Cq, cq0, ("cq", "q_assign", "q_perm", "q_offsets")),
+                              (K, p.Ck, ck0, ("ck", "k_assign", "k_perm", "k_offsets"))):
+        staged = ig.cluster(X, C, 2, p2, init=init)
+        for name, ref in zip(names, staged):
+            assert torch.equal(it1[name], ref), name
+    O2 = ig.forward(Q, K, V, p2, workspace=ws0, cq_init=it0["cq"], ck_init=it0["ck"])  # aliased init
+    assert torch.equal(O2, O1)
+    ig.device_status()
+
+
 def test_forward_host_pipeline_equals_forward():
     """instagen_forward_host (host buffers, head chunks pipelined over three
     streams) gives exactly the device-buffer call's output: every head draws
