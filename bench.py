@@ -47,6 +47,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="budget sweep (error vs dense SDPA and ms per call per budget, one JSON line "
+                         "each) and a warm-started call; not part of the default run")
     return ap.parse_args()
 
 
@@ -218,6 +221,8 @@ def main():
     sample = w.sample_frac if args.sample is None else args.sample
     if args.impl == "reference":
         return reference_arm(args, w, exact, sample)
+    if args.sweep:
+        return sweep_mode(args, w)
 
     import torch
     import block_sparse_attention_head_b200 as ig
@@ -426,6 +431,57 @@ def main():
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def sweep_mode(args, w):
+    """Budget sweep on one GPU: for each (exact, sample) share, ms per call and
+    the relative L2 error of O against dense attention (torch SDPA on the same
+    bf16 inputs); exact-only calls at the same key share for comparison; and a
+    call warm-started from the previous call's centroids with 2 k-means
+    iterations instead of 10."""
+    import torch
+    import torch.nn.functional as F
+    import block_sparse_attention_head_b200 as ig
+    from block_sparse_attention_head_b200 import build, workloads
+    build.build()
+    ig.lib()
+    dev = torch.device("cuda", 0)
+    Q, K, V = workloads.make_inputs(w, device=dev)
+    scale = 1.0 / math.sqrt(w.d)
+    D = F.scaled_dot_product_attention(Q, K, V, scale=scale).float()
+    dn = float(D.pow(2).sum().sqrt())
+
+    def run(exact, sample, iters=w.iters, init=None):
+        p = ig.make_params(w.B, w.H, w.N, w.d, w.Cq, w.Ck, iters=iters, exact_frac=exact, sample_frac=sample,
+                           seed=7, layer=0)
+        ws = torch.empty(ig.workspace_size(p), dtype=torch.uint8, device=dev)
+        O = torch.empty_like(Q)
+        kw = {} if init is None else dict(cq_init=init[0], ck_init=init[1])
+        for _ in range(2):
+            ig.forward(Q, K, V, p, workspace=ws, out=O, **kw)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(3):
+            ig.forward(Q, K, V, p, workspace=ws, out=O, **kw)
+        e1.record()
+        torch.cuda.synchronize()
+        ig.device_status()
+        err = float((O.float() - D).pow(2).sum().sqrt()) / dn
+        it = ig.forward_intermediates(ws, p)
+        return e0.elapsed_time(e1) / 3, err, (it["cq"].clone(), it["ck"].clone())
+
+    for ex, sa in ((0.04, 0.04), (0.08, 0.08), (0.16, 0.16), (0.32, 0.32), (0.08, 0.0), (0.16, 0.0),
+                   (0.32, 0.0), (0.64, 0.0)):
+        ms, err, _ = run(ex, sa)
+        print(json.dumps({"workload": w.name, "exact_frac": ex, "sample_frac": sa, "ms_per_call": round(ms, 3),
+                          "rel_l2_vs_dense": round(err, 4), "kmeans_iters": w.iters}))
+    ms, err, cent = run(0.16, 0.16)
+    ms_w, err_w, _ = run(0.16, 0.16, iters=2, init=cent)
+    print(json.dumps({"workload": w.name, "exact_frac": 0.16, "sample_frac": 0.16, "cold_ms": round(ms, 3),
+                      "cold_rel_l2": round(err, 4), "cold_iters": w.iters, "warm_ms": round(ms_w, 3),
+                      "warm_rel_l2": round(err_w, 4), "warm_iters": 2,
+                      "warm_init": "centroids of the previous call on the same inputs"}))
 
 
 if __name__ == "__main__":
