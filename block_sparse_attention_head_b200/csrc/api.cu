@@ -160,7 +160,7 @@ int select_impl(const float* cq, const float* ck, const int32_t* k_offsets, cons
   if ((rc = check_clusters(p->Cq)) || (rc = check_clusters(p->Ck))) return rc;
   if ((rc = check_budgets(p))) return rc;
   const long long m = budget(p->sample_frac, p->N);
-  if (!cq || !ck || !k_offsets || !exact_groups || !counts) return IG_ERR_INVALID_ARG;
+  if (!cq || !ck || !k_offsets || !exact_groups || !counts || !aligned16(ck)) return IG_ERR_INVALID_ARG;
   if (m > 0 && (!sample_pos || !sample_bias)) return IG_ERR_INVALID_ARG;
   ig::SelectArgs a;
   a.cq = cq;

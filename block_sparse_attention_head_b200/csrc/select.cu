@@ -108,7 +108,10 @@ __global__ void __launch_bounds__(kSelThreads)
   float* S = reinterpret_cast<float*>(wtot + 32);                             // [Ck]
   uint32_t* qw = reinterpret_cast<uint32_t*>(S + a.Ck);                       // [Ck]
   int* koff = reinterpret_cast<int*>(qw + a.Ck);                              // [Ck+1]
-  float* cqrow = reinterpret_cast<float*>(koff + a.Ck + 1);                   // [d]
+  float* lq = reinterpret_cast<float*>(koff + a.Ck + 1);                      // [Ck] logf(q_j)
+  float* cqrow = lq + a.Ck;                                                   // [d]
+  unsigned long long* qinv = reinterpret_cast<unsigned long long*>(
+      (reinterpret_cast<uintptr_t>(cqrow + a.d) + 7) & ~uintptr_t(7));         // [Ck] floor((2^64-1)/q_j)
   __shared__ int s_nexact, s_nskipped;
   __shared__ unsigned s_smax_bits;
   __shared__ long long s_exact_keys;
@@ -128,10 +131,19 @@ __global__ void __launch_bounds__(kSelThreads)
   __syncthreads();
 
   // (b) scores: fp32 fused multiply-add chain over k = 0..d-1, then * scale
+  // (the row is fetched 32 values at a time with 16-byte loads, all in
+  // flight together, ahead of the serial fma chain)
   for (int j = tid; j < Ck; j += kSelThreads) {
-    const float* ckr = a.ck + ((size_t)bh * Ck + j) * d;
+    const float4* ckr = reinterpret_cast<const float4*>(a.ck + ((size_t)bh * Ck + j) * d);
     float acc = 0.0f;
-    for (int k = 0; k < d; ++k) acc = __fmaf_rn(cqrow[k], __ldg(ckr + k), acc);
+    for (int k0 = 0; k0 < d; k0 += 32) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(ckr + k0 / 4 + u);
+      const float* f = reinterpret_cast<const float*>(v);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) acc = __fmaf_rn(cqrow[k0 + e], f[e], acc);
+    }
     S[j] = __fmul_rn(acc, a.scale);
   }
   __syncthreads();
@@ -201,6 +213,8 @@ __global__ void __launch_bounds__(kSelThreads)
     uint32_t q = 0u;
     if (qw[j]) q = (a.mode == 1) ? 1u : group_weight(S[j], smax);
     qw[j] = q;
+    lq[j] = logf((float)q);  // the draws' log-weights take it from here
+    qinv[j] = q ? ~0ull / q : 0ull;
     cdf[j] = (unsigned long long)(koff[j + 1] - koff[j]) * q;
   }
   __syncthreads();
@@ -233,9 +247,14 @@ __global__ void __launch_bounds__(kSelThreads)
         raise_error(kErrSampling);
       } else {
         const unsigned long long start = cdf[j] - (unsigned long long)(koff[j + 1] - koff[j]) * q;
-        const unsigned long long o = (r - start) / q;
+        // floor((r - start) / q) by the group's reciprocal: with
+        // qinv = floor((2^64-1)/q) and x < 2^56, mulhi(x, qinv) is the
+        // quotient or one less; one remainder test makes it exact
+        const unsigned long long x = r - start;
+        unsigned long long o = __umul64hi(x, qinv[j]);
+        if (x - o * q >= q) ++o;
         pos = koff[j] + (int32_t)o;
-        bias = logT - logf((float)q) - logm;
+        bias = logT - lq[j] - logm;
       }
     }
     a.sample_pos[gi * m + t] = pos;
@@ -251,8 +270,8 @@ __global__ void __launch_bounds__(kSelThreads)
 cudaError_t launch_select_sample(const SelectArgs& a, cudaStream_t s) {
   int p2 = 1;
   while (p2 < a.Ck) p2 <<= 1;
-  const size_t sm = (size_t)p2 * 8 + (size_t)a.Ck * 8 + 32 * 8 + (size_t)a.Ck * 4 * 2 + (size_t)(a.Ck + 1) * 4 +
-                    (size_t)a.d * 4 + 16;
+  const size_t sm = (size_t)p2 * 8 + (size_t)a.Ck * 8 + 32 * 8 + (size_t)a.Ck * 4 * 3 + (size_t)(a.Ck + 1) * 4 +
+                    (size_t)a.d * 4 + 8 + (size_t)a.Ck * 8 + 16;
   cudaError_t e = cudaFuncSetAttribute(select_sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   dim3 grid(a.Cq, a.BH);

@@ -164,7 +164,8 @@ int instagen_gather(const void* X, const int32_t* perm, const instagen_params* p
  *   and the remaining keys are represented by a sample drawn in proportion to
  *   their estimated attention and reweighted by inverse sampling
  *   probability"; Figure 3 (b), (c)).
- *   cq [B,H,Cq,d] fp32, ck [B,H,Ck,d] fp32 centroids; k_offsets [B,H,Ck+1].
+ *   cq [B,H,Cq,d] fp32, ck [B,H,Ck,d] fp32 centroids (ck 16-byte aligned);
+ *   k_offsets [B,H,Ck+1].
  *   Score S_ij = fp32 fused-multiply-add chain of cq_i . ck_j over k = 0..d-1,
  *   then one fp32 multiply by softmax_scale (bit-reproducible).
  *   Exact set of query group i: non-empty key groups ranked by S_ij descending
