@@ -257,13 +257,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
     // warp's 64 rows, from the row positions held by lanes (posA: rows 0-31,
     // posB: rows 32-63)
     const uint32_t lane_dst = (uint32_t)((ch >> 3) * 16384);
+    // All row positions are fetched from their lanes first (independent
+    // shuffles, latencies overlapped), then the copies are issued back to
+    // back.
     auto issue_rows = [&](const auto* base, uint32_t dst, int posA, int posB) {
       const auto* head = base + (size_t)bh * N * D + ch * 8;
-#pragma unroll 4
-      for (int i = 0; i < 64 / kRpi; ++i) {
-        const int rl = i * kRpi + rsub;
-        const int p = __shfl_sync(0xffffffffu, i * kRpi < 32 ? posA : posB, rl & 31);
-        const int r = 64 * pw + rl;
+      constexpr int kIters = 64 / kRpi;
+      int pr[kIters];
+#pragma unroll
+      for (int i = 0; i < kIters; ++i)
+        pr[i] = __shfl_sync(0xffffffffu, i * kRpi < 32 ? posA : posB, (i * kRpi + rsub) & 31);
+#pragma unroll
+      for (int i = 0; i < kIters; ++i) {
+        const int r = 64 * pw + i * kRpi + rsub;
+        const int p = pr[i];
         cp_async_16(dst + lane_dst + sw128_offset(r, ch & 7), head + (size_t)(p < 0 ? 0 : p) * D,
                     p < 0 ? 0u : 16u);
       }
