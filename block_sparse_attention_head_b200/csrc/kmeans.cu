@@ -1,6 +1,6 @@
 // Batched k-means for the query / key clustering of InstaGen (thelatestinai.com
-// paper page, Figure 3 (a): "queries and keys are clustered into groups";
-// Figure 2 caption: Cq = 100, Ck = 500).
+// paper page, Figure 3 (a): both the queries and the keys are partitioned by
+// clustering; Figure 2 caption: Cq = 100, Ck = 500).
 //
 // One Lloyd iteration = assign (tensor cores) -> stable counting sort ->
 // deterministic per-cluster mean.  Distances: ||x - c||^2 = ||x||^2 + ||c||^2

@@ -1,8 +1,9 @@
-// Semantic permutation (InstaGen abstract: "a semantically permuted attention
-// matrix"; Figure 3 (d): "queries in a group share the same keys, so attention
-// runs over dense blocks").  A stable counting sort puts every cluster in a
-// contiguous range of slots, and a row gather copies K and V into that order
-// with 128-bit coalesced loads and stores.
+// Semantic permutation (InstaGen abstract: tokens are reordered by cluster so
+// the attention matrix becomes block structured; Figure 3 (d): a query group
+// attends to one common key list, which makes the work dense tiles).  A stable
+// counting sort puts every cluster in a contiguous range of slots, and a row
+// gather copies K and V into that order with 128-bit coalesced loads and
+// stores.
 #include "internal.cuh"
 #include "ptx.cuh"
 

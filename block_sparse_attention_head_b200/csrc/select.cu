@@ -1,9 +1,9 @@
 // Centroid scoring, exact set and group-shared importance sampling
-// (InstaGen abstract: "the top-scoring keys form an exact set that is computed
-// in full and the remaining keys are represented by a sample drawn in
-// proportion to their estimated attention and reweighted by inverse sampling
-// probability ... Each query cluster draws one sample shared by all its
-// queries"; thelatestinai.com paper page, Figure 3 (b), (c)).
+// (InstaGen abstract: the highest-scoring keys are attended exactly, the rest
+// are stood in for by a sample whose draw probability follows the estimated
+// attention and whose scores are weighted by the inverse of that probability;
+// one sample per query cluster, used by all of its queries; thelatestinai.com
+// paper page, Figure 3 (b), (c)).
 //
 // Everything that decides an index is integer arithmetic or a correctly
 // rounded fp32 operation in a fixed order (fused multiply-add chain for the

@@ -6,12 +6,13 @@
  * Method (InstaGen: Group-Shared Importance Sampling for Fast Video
  * Generation, arXiv 2611.08610; abstract, and Figure 3 (a)-(d) of the
  * thelatestinai.com paper page).  Per head:
- *   (a) queries and keys are clustered into Cq and Ck groups (k-means) and
- *       permuted so that every group is a contiguous block;
- *   (b) centroid scores give each query group a probability pi over the key
- *       groups;
- *   (c) the top-scoring key groups form an exact set (the top group is always
- *       kept); the remaining keys are covered by m draws in proportion to pi,
+ *   (a) k-means splits the queries into Cq groups and the keys into Ck
+ *       groups, and a permutation makes every group a contiguous block;
+ *   (b) from centroid scores each query group gets a probability pi over
+ *       the key groups;
+ *   (c) the best-ranked key groups make up an exact set (never empty: the
+ *       first-ranked group is in it); the remaining keys are covered by m
+ *       draws in proportion to pi,
  *       one list shared by every query of the group, each draw carrying the
  *       log-weight log(1/(pi*m));
  *   (d) exact blocks and sampled keys go through one online-softmax kernel.
@@ -67,8 +68,8 @@ typedef struct {
 } instagen_params;
 
 /* E and m for these parameters: the share times N rounded to nearest, halves
- * away from zero (Table 1 caption: "E + S", the exact and sampled shares of
- * keys per sparse call). */
+ * away from zero (Table 1 caption: E + S denotes the fraction of keys attended
+ * exactly plus the fraction sampled, per sparse call). */
 int64_t instagen_exact_budget(const instagen_params* p);
 int64_t instagen_sample_budget(const instagen_params* p);
 
@@ -89,7 +90,7 @@ int instagen_device_status(void* stream);
 
 /*
  * (a) k-means clustering + stable permutation of one tensor X (Q or K),
- *     Figure 3 (a); "semantically permuted attention matrix" (abstract).
+ *     Figure 3 (a); the abstract's reordering of tokens by cluster.
  *   X         [B,H,N,d] bf16.
  *   C         cluster count, 1 <= C <= 4096.
  *   iters     Lloyd iterations >= 1 (each: assign to the nearest centroid by
@@ -160,10 +161,10 @@ int instagen_gather(const void* X, const int32_t* perm, const instagen_params* p
 
 /*
  * (b)+(c) Centroid scores, exact set and the group-shared sample
- *   (abstract: "top-scoring keys form an exact set that is computed in full
- *   and the remaining keys are represented by a sample drawn in proportion to
- *   their estimated attention and reweighted by inverse sampling
- *   probability"; Figure 3 (b), (c)).
+ *   (abstract: the highest-scoring keys are attended exactly and the others
+ *   through a sample drawn with probability following their estimated
+ *   attention, weighted by the inverse of that probability; Figure 3 (b),
+ *   (c)).
  *   cq [B,H,Cq,d] fp32, ck [B,H,Ck,d] fp32 centroids (ck 16-byte aligned);
  *   k_offsets [B,H,Ck+1].
  *   Score S_ij = fp32 fused-multiply-add chain of cq_i . ck_j over k = 0..d-1,
@@ -191,8 +192,8 @@ int instagen_select_sample(const float* cq, const float* ck, const int32_t* k_of
 
 /*
  * (d) Sparse attention over exact blocks plus the weighted sample, one
- *   online-softmax pass (Figure 3 (d); "computes them together with the top-k
- *   blocks in a single attention kernel", ICLR listing abstract).
+ *   online-softmax pass (Figure 3 (d); ICLR listing abstract: the sampled keys
+ *   and the top-k blocks are processed by the same attention kernel).
  *   Q  [B,H,N,d] bf16 in ORIGINAL token order (rows gathered via q_perm).
  *   Kp [B,H,N,d] bf16 and Vp [B,H,N,d] fp16, both in key-cluster (permuted)
  *   order (instagen_gather with to_f16 = 0 and 1).

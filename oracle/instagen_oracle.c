@@ -10,23 +10,24 @@
  * Sources (web pages on "InstaGen: Group-Shared Importance Sampling for Fast
  * Video Generation", arXiv 2611.08610):
  *   [ABS]   the paper's abstract (paper-reading aggregator page and the
- *           thelatestinai.com paper page): block selection cast as importance
- *           sampling; top-scoring keys form an exact set computed in full; the
- *           remaining keys are a sample drawn in proportion to their estimated
- *           attention and reweighted by inverse sampling probability; one
- *           sample per query cluster shared by all of its queries.
- *   [FIG3]  thelatestinai.com paper page, Figure 3 caption: (a) queries and
- *           keys are clustered into groups; (b) centroid scores give each key
- *           group a probability pi for each query group; (c) the top key group
- *           is always kept, the rest are sampled in proportion to pi and
- *           weighted by 1/pi; (d) queries of a group share keys, so attention
- *           runs over dense blocks in one kernel.
+ *           thelatestinai.com paper page): block selection treated as an
+ *           importance-sampling problem; the highest-scoring keys are attended
+ *           exactly; the others enter through a sample whose draw probability
+ *           follows their estimated attention, each sampled score weighted by
+ *           the inverse of that probability; one sample per query cluster,
+ *           used by every query in it.
+ *   [FIG3]  thelatestinai.com paper page, Figure 3 caption: (a) clustering
+ *           of both queries and keys; (b) from centroid scores, a probability
+ *           pi per key group for each query group; (c) the first-ranked key
+ *           group is never dropped, the other keys are drawn with probability
+ *           following pi and weighted by 1/pi; (d) one key list per query
+ *           group, so a single kernel works on dense tiles.
  *   [FIG2]  same page, Figure 2 caption: SVG2 clustering configuration
  *           Cq = 100 query and Ck = 500 key clusters.
- *   [ICLR]  acceptodds.com ICLR 2027 listing, abstract: the sample is shared
- *           across all queries of the cluster and computed together with the
- *           top-k blocks in one attention kernel, sampled scores reweighted
- *           to stand for the whole skipped region.
+ *   [ICLR]  acceptodds.com ICLR 2027 listing, abstract: every query of the
+ *           cluster uses the same sample; sampled keys and top-k blocks go
+ *           through one attention kernel, and the weights on the sampled
+ *           scores make them represent all of the skipped keys.
  *
  * Where the pages are silent the plainest reading is taken; each such reading
  * is marked "[reading]" below.
@@ -83,7 +84,8 @@ void orc_philox_batch(int64_t n, const uint32_t* ctrs, const uint32_t* keys, uin
 /* ------------------------------------------------------------------------- */
 /* Budgets.  [reading] E and m are the given shares of the N keys rounded to
  * the nearest integer, halves away from zero (Table 1 caption of the paper
- * page: "E + S", exact and sampled share of keys per sparse call).           */
+ * page: E + S names the exactly attended plus the sampled key fraction of a
+ * sparse call).                                                              */
 /* ------------------------------------------------------------------------- */
 int64_t orc_budget(float frac, int64_t N)
 {
@@ -172,8 +174,7 @@ int orc_kmeans(const float* X, int64_t N, int d, int C, int iters, const float* 
 }
 
 /* ------------------------------------------------------------------------- */
-/* Semantic permutation [ABS "semantically permuted attention matrix",
- * FIG3 (d)].  [reading] stable counting sort by cluster id: cluster j owns
+/* Semantic permutation [ABS: tokens reordered by cluster; FIG3 (d)].  [reading] stable counting sort by cluster id: cluster j owns
  * the contiguous range [offsets[j], offsets[j+1]); inside it tokens keep
  * ascending original index.  perm[p] = original index at permuted slot p.    */
 /* ------------------------------------------------------------------------- */
@@ -210,8 +211,8 @@ void orc_scores(const float* cq, int Cq, const float* ck, int Ck, int d, float s
 }
 
 /* ------------------------------------------------------------------------- */
-/* Integer sampling weight of a skipped key group [ABS "drawn in proportion to
- * their estimated attention"; FIG3 (b),(c)].
+/* Integer sampling weight of a skipped key group [ABS: draw probability
+ * follows the estimated attention; FIG3 (b),(c)].
  * [reading] the estimated attention of every key of group j, seen from query
  * group i, is exp(S_ij); the group's mass is |K_j| exp(S_ij), so a key's
  * probability is proportional to q_j ~ 2^24 * exp(S_ij - Smax).  It is held
@@ -260,8 +261,8 @@ uint32_t orc_group_weight(float s, float smax)
 /* ------------------------------------------------------------------------- */
 /* (c) Exact set, pi and the group-shared sample for one query group i.
  *
- * Exact set [ABS "top-scoring keys form an exact set that is computed in
- * full"; FIG3 (c) "the top key group is always kept"].  [reading] non-empty
+ * Exact set [ABS: the best-scoring keys are attended exactly; FIG3 (c): the
+ * first-ranked key group is never dropped].  [reading] non-empty
  * key groups ranked by S_ij descending (ties: lowest j); the rank-0 group is
  * always taken; the next groups are taken while the running key count stays
  * <= E, stopping at the first group that does not fit (a prefix of the
@@ -276,8 +277,8 @@ uint32_t orc_group_weight(float s, float smax)
  * key offset in it is (r - CDF_{j-1}) / q_j (integer division: uniform inside
  * the group).  The key's probability is p = q_j / T, and its log-weight is
  * log(1/(p m)) = ln T - ln q_j - ln m, which is added to its logit so that
- * the m draws stand for the whole skipped region (ICLR "reweighted to account
- * for the full skipped region").  No skipped keys -> no draws.
+ * the m draws stand for the whole skipped region (ICLR: the weights make the
+ * sample represent every skipped key).  No skipped keys -> no draws.
  *
  * Uniform variant (mode 1; Figure 2/4/5 captions run "uniform" sampling):
  * q_j = 1 for every skipped group.

@@ -408,7 +408,7 @@ def test_attention_rows_counts_duplicates(oracle_mod):
 def test_error_falls_with_sample_size(oracle_mod):
     """The tiny configuration (N=4096, d=64, Cq=16, Ck=64, exact 8%) runs in
     seconds; its error against dense attention falls as the sample grows
-    (ICLR listing: reconstruction error decreases as more tokens are sampled;
+    (ICLR listing: the reconstruction error shrinks as the sample grows;
     an i.i.d. estimator's error shrinks like 1/sqrt(m)), and importance
     sampling beats uniform at every size (Figure 4 caption)."""
     w = workloads.TINY
