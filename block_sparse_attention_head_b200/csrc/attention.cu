@@ -1,31 +1,38 @@
 // Sparse attention over the exact key groups plus the group-shared weighted
 // sample, in one online-softmax pass (InstaGen, thelatestinai.com paper page,
-// Figure 3 (d): "queries in a group share the same keys, so attention runs
-// over dense blocks in one kernel"; ICLR listing abstract: the sample is
-// "computed together with the top-k blocks in a single attention kernel, with
-// sampled scores reweighted to account for the full skipped region").
+// Figure 3 (d): every query of a group attends to one common key list, so the
+// work is dense tiles; ICLR listing abstract: the sampled keys run in the same
+// kernel as the top-k blocks, their scores carrying a weight that stands for
+// the part of the skipped region they represent).
 //
 // CTA = two tiles of 128 queries (Q0, Q1) of one query group, gathered from Q
 // through the query permutation.  Both share the group's key list: its exact
 // groups (rank order; contiguous ranges of the permuted K/V) followed by its m
-// sample slots (gathered rows with log-weight), walked in tiles of 128 keys.
+// sample slots (gathered rows with log-weight w), walked in tiles of 128 keys.
 // Per key tile j and query tile t:
-//   S_t = Q_t K_j^T        tcgen05 (M=128, N=128, K=d, bf16), fp32 in TMEM
-//   P_t = 2^(S_t*scale*log2e + bias*log2e - m_t)    softmax warpgroup t,
-//                          written back as fp16 into S_t's TMEM columns
+//   S_t = Q_t K_j^T + 1 w_j^T/scale    tcgen05 (M=128, N=128, bf16), fp32 in
+//                          TMEM: d/16 steps over Q and K plus one side step
+//                          whose 16-column operands hold (1, 1) per query row
+//                          and (w_hi, w_lo) per key slot (w/scale in two bf16
+//                          terms; -inf for padding slots, 0 for exact keys)
+//   P_t = 2^(S_t*scale*log2e - m_t)    softmax warpgroup t, written back as
+//                          fp16 into S_t's TMEM columns
 //   O_t += P_t V_j         tcgen05 with A (P_t) read from TMEM, fp16 operands
-// The tensor pipe alternates [PV_0(j-1), S_0(j)] and [PV_1(j-1), S_1(j)], so
-// one warpgroup's softmax runs while the other tile's MMAs execute.  The
-// running max is only raised when it grows by more than 8 (log2 units), so
-// P <= 256 and the O rescale (a TMEM read-modify-write) is rare; it is done by
-// the softmax warpgroup after S_t(j) lands, which the MMA pipe orders after
-// PV_t(j-1).  P and V are fp16 (V converted by the gather): 11 mantissa bits
-// keep the output within 2e-3 mean relative error after its bf16 rounding.
+// Folding w into the product leaves the softmax one code path with no
+// per-column loads.  The tensor pipe alternates [PV_0(j-1), S_0(j)] and
+// [PV_1(j-1), S_1(j)], so one warpgroup's softmax runs while the other tile's
+// MMAs execute.  The running max is only raised when it grows by more than 8
+// (log2 units), so P <= 256 and the O rescale (a TMEM read-modify-write) is
+// rare; it is done by the softmax warpgroup after S_t(j) lands, which the MMA
+// pipe orders after PV_t(j-1).  P and V are fp16 (V converted by the gather):
+// 11 mantissa bits keep the output within 2e-3 mean relative error after its
+// bf16 rounding.
 //
 // Warps: 0 MMA issuer + TMEM owner, 1 idle, 2-3 producer (cp.async 16-byte
 // row gathers into the 128-byte-swizzled operand layout, completion tracked
-// by the stage mbarriers so the producer never blocks on memory), 4-7
-// softmax for Q0, 8-11 softmax for Q1 (thread = query row = TMEM lane).
+// by the stage mbarriers so the producer never blocks on memory; the key side
+// rows are plain shared stores), 4-7 softmax for Q0, 8-11 softmax for Q1
+// (thread = query row = TMEM lane).
 #include "internal.cuh"
 #include "ptx.cuh"
 
@@ -46,10 +53,14 @@ struct AttnSmem {
   static constexpr int kQ = 0;                          // 2 query tiles
   static constexpr int kK = kQ + 2 * kTileBytes;        // 2 stages
   static constexpr int kV = kK + 2 * kTileBytes;        // 2 stages
-  static constexpr int kGStart = kV + 2 * kTileBytes;   // exact group start slots
-  static constexpr int kGPre = kGStart + kAttnMaxExactGroups * 4;         // exclusive prefix of sizes
-  static constexpr int kBias = kGPre + (kAttnMaxExactGroups + 1) * 4 + 12;  // 8 warps x 2 x 128 fp32
-  static constexpr int kBars = kBias + 8 * 2 * 128 * 4;
+  // 16-column side blocks of the S product (no swizzle, 128 rows x 32 bytes):
+  // ones for the query tiles, the slot log-weight over the scale for K
+  static constexpr int kSideBytes = 128 * 32;
+  static constexpr int kQx = kV + 2 * kTileBytes;             // shared by both query tiles
+  static constexpr int kKx = kQx + kSideBytes;                // 2 stages
+  static constexpr int kGStart = kKx + 2 * kSideBytes;        // exact group start slots
+  static constexpr int kGPre = kGStart + kAttnMaxExactGroups * 4;  // exclusive prefix of sizes
+  static constexpr int kBars = (kGPre + (kAttnMaxExactGroups + 1) * 4 + 15) / 16 * 16;
   static constexpr int kNumBars = 16;
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kBytes = kMisc + 64;
@@ -70,7 +81,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   int* gstart = reinterpret_cast<int*>(smem + L::kGStart);
   int* gpre = reinterpret_cast<int*>(smem + L::kGPre);
-  float* bias_s = reinterpret_cast<float*>(smem + L::kBias);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;   // [2] stages
@@ -167,9 +177,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
     if (lane == 0) gpre[n_exact] = run;
   }
   if (tid == 32) {
-    mbar_init(q_full, kProducers);
+    // producers arrive twice per phase: their copies (cp.async) and their
+    // side-block stores
+    mbar_init(q_full, 2 * kProducers);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&k_full[s], kProducers);
+      mbar_init(&k_full[s], 2 * kProducers);
       mbar_init(&v_full[s], kProducers);
       mbar_init(&k_empty[s], 1);
       mbar_init(&v_empty[s], 1);
@@ -195,6 +207,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
   const uint32_t q_s = smem_u32(smem + L::kQ);
   const uint32_t k_s = smem_u32(smem + L::kK);
   const uint32_t v_s = smem_u32(smem + L::kV);
+  const uint32_t qx_s = smem_u32(smem + L::kQx);
+  const uint32_t kx_s = smem_u32(smem + L::kKx);
   const int32_t* spos = a.sample_pos + grp * (size_t)a.m;
   const float* sbias = a.sample_bias + grp * (size_t)a.m;
 
@@ -224,6 +238,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
         cp_async_16(dst + (c >> 3) * 16384 + sw128_offset(rr, c & 7), src + c * 8, valid ? 16u : 0u);
     }
     cp_async_arrive_noinc(q_full);
+    // Side blocks: row r of the query side is (1, 1, 0, ...), row r of a key
+    // side is (w_hi, w_lo, 0, ...) with w_hi + w_lo = log-weight / scale in
+    // two bf16 terms, so one more K=16 step of the S product adds the slot's
+    // log-weight (and -inf for padding slots) to every score of its column.
+    // Only the first 16 bytes of a key side row change per tile; this thread
+    // owns rows tp and tp + 64 of every side block.
+    auto side_off = [](int r, int chunk) -> uint32_t {
+      return (uint32_t)((r >> 3) * 256 + chunk * 128 + (r & 7) * 16);
+    };
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = tp + 64 * h;
+      st_shared_v4(qx_s + side_off(r, 0), 0x3F803F80u, 0u, 0u, 0u);  // bf16 1.0, 1.0
+      st_shared_v4(qx_s + side_off(r, 1), 0u, 0u, 0u, 0u);
+      st_shared_v4(kx_s + side_off(r, 1), 0u, 0u, 0u, 0u);
+      st_shared_v4(kx_s + L::kSideBytes + side_off(r, 1), 0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(q_full);
+    const float inv_scale = kLog2e / a.scale_log2;
+    // slot log-weight over the scale: 0 for exact keys, -inf past the list
+    auto slot_w = [&](int j, int r) -> float {
+      const int l = j * 128 + r;
+      if (l < Xi) return 0.f;
+      if (l < Lk) return __ldg(sbias + (l - Xi)) * inv_scale;
+      return -__int_as_float(0x7f800000);
+    };
+    auto side_row = [&](uint32_t base, int r, float w) {
+      const float hi = __bfloat162float(__float2bfloat16_rn(w));
+      const float lo = isfinite(w) ? w - hi : 0.f;
+      st_shared_v4(base + side_off(r, 0), pack_bf16x2(hi, lo), 0u, 0u, 0u);
+    };
     // Warp w of the producer owns rows [64w, 64w+64) of every K/V tile; lane l
     // resolves the permuted key positions of rows 64w+l and 64w+32+l (one tile
     // ahead, since sample positions come from global memory).  The copies are
@@ -276,15 +322,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
       }
     };
     int eA = 0, eB = 0;  // exact-group cursors of the two row streams
-    int nA = key_pos(0, 64 * pw + lane, eA), nB = key_pos(0, 64 * pw + 32 + lane, eB);
+    const int rA = 64 * pw + lane, rB = 64 * pw + 32 + lane;
+    int nA = key_pos(0, rA, eA), nB = key_pos(0, rB, eB);
+    float wA = slot_w(0, rA), wB = slot_w(0, rB);
     for (int kt = 0; kt < ntk; ++kt) {
       const int s = kt & 1, use = kt >> 1;
       const int posA = checked(nA), posB = checked(nB);
+      const float cwA = wA, cwB = wB;
       if (kt + 1 < ntk) {
-        nA = key_pos(kt + 1, 64 * pw + lane, eA);
-        nB = key_pos(kt + 1, 64 * pw + 32 + lane, eB);
+        nA = key_pos(kt + 1, rA, eA);
+        nB = key_pos(kt + 1, rB, eB);
+        wA = slot_w(kt + 1, rA);
+        wB = slot_w(kt + 1, rB);
       }
       if (kt >= 2 && !mbar_wait(&k_empty[s], (use - 1) & 1, abort_flag)) break;
+      side_row(kx_s + s * L::kSideBytes, rA, cwA);
+      side_row(kx_s + s * L::kSideBytes, rB, cwB);
+      fence_proxy_async_smem();
+      mbar_arrive(&k_full[s]);
       issue_rows(a.Kp, k_s + s * L::kTileBytes, posA, posB);
       cp_async_arrive_noinc(&k_full[s]);
       if (kt >= 2 && !mbar_wait(&v_empty[s], (use - 1) & 1, abort_flag)) break;
@@ -303,64 +358,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
     float m_run = -__int_as_float(0x7f800000);
     float l_run = 0.f;
     bool ok = active;
-    // column log-weights (log2 units) of key tile j, lane's 4 columns; loaded
-    // one tile ahead so the global-load latency stays off the critical path
-    auto load_bias = [&](int j, float* b) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int l = j * 128 + lane * 4 + e;
-        if (l < Xi)
-          b[e] = 0.f;
-        else if (l < Lk)
-          b[e] = __ldg(sbias + (l - Xi));
-        else
-          b[e] = -__int_as_float(0x7f800000);
-      }
-    };
-    float bnext[4];
-    if (ok) load_bias(0, bnext);
     for (int kt = 0; kt < ntk && ok; ++kt) {
-      // this warp's private copy of the tile's column log-weights
-      float* wb = bias_s + ((warp - 4) * 2 + (kt & 1)) * 128;
-      *reinterpret_cast<float4*>(wb + lane * 4) =
-          make_float4(bnext[0] * kLog2e, bnext[1] * kLog2e, bnext[2] * kLog2e, bnext[3] * kLog2e);
-      if (kt + 1 < ntk) load_bias(kt + 1, bnext);
-      __syncwarp();
       if (!mbar_wait_warp(&s_full[t], kt & 1, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      // the whole S row of this thread in registers: one TMEM round trip
+      // the whole S row of this thread in registers: one TMEM round trip; S
+      // already carries the column log-weights (side step of the product)
       float x[128];
       tmem_ld32(s_col + 0, x);
       tmem_ld32(s_col + 32, x + 32);
       tmem_ld32(s_col + 64, x + 64);
       tmem_ld32(s_col + 96, x + 96);
       tmem_wait_ld();
-      // all-exact tiles carry no log-weight and no padding: scale after the max
-      const bool plain = kt * 128 + 128 <= Xi;
       float mxp[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) mxp[e] = -__int_as_float(0x7f800000);
-      if (plain) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mxp[c & 3] = fmaxf(mxp[c & 3], x[c]);
-      } else {
-        const float4* b4 = reinterpret_cast<const float4*>(wb);
-#pragma unroll
-        for (int c = 0; c < 128; c += 4) {
-          const float4 bb = b4[c >> 2];
-          x[c + 0] = fmaf(x[c + 0], a.scale_log2, bb.x);
-          x[c + 1] = fmaf(x[c + 1], a.scale_log2, bb.y);
-          x[c + 2] = fmaf(x[c + 2], a.scale_log2, bb.z);
-          x[c + 3] = fmaf(x[c + 3], a.scale_log2, bb.w);
-          mxp[(c >> 2) & 1] = fmaxf(mxp[(c >> 2) & 1], fmaxf(x[c], x[c + 1]));
-          mxp[((c >> 2) & 1) + 2] = fmaxf(mxp[((c >> 2) & 1) + 2], fmaxf(x[c + 2], x[c + 3]));
-        }
-      }
-      float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
-      if (plain) mx *= a.scale_log2;  // scale > 0
+      for (int c = 0; c < 128; ++c) mxp[c & 3] = fmaxf(mxp[c & 3], x[c]);
+      // scale after the max (scale > 0)
+      const float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])) * a.scale_log2;
       const float m_new = fmaxf(m_run, mx);
       const bool rescale = m_new > m_run + kRescaleThreshold;
       float alpha = 1.f;
@@ -377,8 +395,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const int c = c4 * 32 + e;
-          const float p0 = ex2_approx(plain ? fmaf(x[c], a.scale_log2, neg_m) : x[c] + neg_m);
-          const float p1 = ex2_approx(plain ? fmaf(x[c + 1], a.scale_log2, neg_m) : x[c + 1] + neg_m);
+          const float p0 = ex2_approx(fmaf(x[c], a.scale_log2, neg_m));
+          const float p1 = ex2_approx(fmaf(x[c + 1], a.scale_log2, neg_m));
           rsp[(e >> 1) & 3] += p0 + p1;
           x[c4 * 16 + (e >> 1)] = __uint_as_float(pack_f16x2(p0, p1));
         }
@@ -478,6 +496,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
             const uint64_t bd = umma_desc_sw128(kb + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
             umma_bf16_ss(tmem + 128 * t, ad, bd, idesc_qk, k > 0 ? 1u : 0u);
           }
+          umma_bf16_ss(tmem + 128 * t, umma_desc_noswz(qx_s, 128, 256),
+                       umma_desc_noswz(kx_s + s * L::kSideBytes, 128, 256), idesc_qk, 1u);
           umma_commit(&s_full[t]);
         }
       }

@@ -359,6 +359,19 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// Shared-memory matrix descriptor, no swizzle, K-major: the operand is tiled
+// in 8-row x 16-byte core matrices (128 contiguous bytes each); lbo = byte
+// distance between core matrices adjacent along K, sbo = between core matrices
+// adjacent along M/N.
+__device__ __forceinline__ uint64_t umma_desc_noswz(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;  // layout type 0 (no swizzle) in bits 61-63
+  return d;
+}
+
 // Instruction descriptor, kind::f16: fp32 accumulator, A and B both bf16
 // (f16_operands = false) or both fp16 (true).
 __host__ __device__ constexpr uint32_t umma_idesc_f16kind(int M, int N, bool a_mn_major, bool b_mn_major,
