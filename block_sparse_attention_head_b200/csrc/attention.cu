@@ -376,7 +376,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
 #pragma unroll
       for (int e = 0; e < 4; ++e) mxp[e] = -__int_as_float(0x7f800000);
 #pragma unroll
-      for (int c = 0; c < 128; ++c) mxp[c & 3] = fmaxf(mxp[c & 3], x[c]);
+      for (int c = 0; c < 128; c += 2) mxp[(c >> 1) & 3] = fmax3(mxp[(c >> 1) & 3], x[c], x[c + 1]);
       // scale after the max (scale > 0)
       const float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])) * a.scale_log2;
       const float m_new = fmaxf(m_run, mx);
