@@ -230,6 +230,10 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   const int nchunks = g.c_pad / g.chunk;
   const int half = g.chunk / 2;         // centroid rows per CTA per chunk
   const int kblocks = 2 * L::kXBlocks;  // hi blocks then lo blocks
+  // A single chunk whose K-blocks all fit in the ring stays resident: it is
+  // loaded once per head (an epoch) into stages 0..kblocks-1 instead of once
+  // per unit, and the MMA issuer waits on it only when the head changes.
+  const bool resident = nchunks == 1 && kblocks <= kAssignStages;
 
   if (tid == 0) {
     for (int s = 0; s < kAssignStages; ++s) {
@@ -266,8 +270,24 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     prefetch_tmap(&tmap_c);
     int st = 0;
     bool ok = true;
+    int ep = -1, cur_bh = -1;  // resident: epoch = head
     for (int i = 0; i < nunits && ok; ++i) {
       const int bh = (int)((u0 + i) / uph);
+      if (resident) {
+        if (bh == cur_bh) continue;
+        cur_bh = bh;
+        ++ep;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (ep >= 1 && !mbar_wait_sleep(&c_empty[kb], (ep - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&c_full[kb], 2 * half * 128);
+          tma_load_2d_pair(st_base + kb * L::kStageBytes, &tmap_c, kb * 64, bh * g.c_pad + (int)rank * half,
+                           mapa_shared(smem_u32(&c_full[kb]), 0));
+        }
+        continue;
+      }
       for (int c = 0; c < nchunks && ok; ++c) {
         for (int kb = 0; kb < kblocks; ++kb, ++st) {
           const int s = st % kAssignStages;
@@ -300,10 +320,39 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     const uint32_t idesc = umma_idesc_bf16(256, g.chunk, false, false);
     int st = 0, gc = 0;  // stage counter, global chunk counter (TMEM buffer phases)
     bool ok = true;
+    int ep = -1, cur_bh = -1;  // resident: epoch = head
     for (int i = 0; i < nunits && ok; ++i) {
       const int buf = i % kAssignXBufs;
       if (!mbar_wait_sleep(&x_full[buf], (i / kAssignXBufs) & 1, abort_flag)) break;
       const uint32_t xb = x_base + buf * L::kXTileBytes;
+      if (resident) {
+        const int bh = (int)((u0 + i) / uph);
+        const bool head_ends = i + 1 == nunits || (int)((u0 + i + 1) / uph) != bh;
+        const int b = gc & 1;
+        if (gc >= 2 && !mbar_wait_sleep(&t_empty[b], ((gc >> 1) - 1) & 1, abort_flag)) break;
+        if (bh != cur_bh) {
+          cur_bh = bh;
+          ++ep;
+          for (int kb = 0; kb < kblocks && ok; ++kb)
+            if (!mbar_wait_sleep(&c_full[kb], ep & 1, abort_flag)) ok = false;
+          if (!ok) break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < kblocks; ++kb) {
+          const int xkb = kb % L::kXBlocks;
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t adesc = umma_desc_sw128(xb + xkb * 16384 + k * 32, 16, 1024);
+            const uint64_t bdesc = umma_desc_sw128(st_base + kb * L::kStageBytes + k * 32, 16, 1024);
+            umma_bf16_ss_pair(tmem + (uint32_t)(b * 256), adesc, bdesc, idesc, (kb | k) != 0);
+          }
+        }
+        if (head_ends)
+          for (int kb = 0; kb < kblocks; ++kb) umma_commit_pair_mc(&c_empty[kb], 3);
+        umma_commit_pair_mc(&t_full[b], 3);
+        ++gc;
+        umma_commit_pair_mc(&x_empty[buf], 3);
+        continue;
+      }
       for (int c = 0; c < nchunks && ok; ++c, ++gc) {
         const int b = gc & 1;
         if (gc >= 2 && !mbar_wait_sleep(&t_empty[b], ((gc >> 1) - 1) & 1, abort_flag)) {
