@@ -441,6 +441,16 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         if (lane == 0) mbar_arrive_cluster(t_empty_lead);
       }
       if (!ok) break;
+      if (nchunks == 1) {
+        // one chunk per unit: the group that reduced it (units alternate
+        // between the groups) holds the whole minimum and writes it, so the
+        // two groups work on consecutive units in parallel
+        if ((gc - 1) % 2 == grp) {
+          const int tok = pr * 256 + (int)rank * 128 + r;
+          if (tok < g.N) assign[(size_t)bh * g.N + tok] = best_j;
+        }
+        continue;
+      }
       // merge the two groups' minima of this unit (slot i & 1); on equal
       // distances the lower centroid index wins
       float2* slot = merge + (i & 1) * 128 + r;
