@@ -71,11 +71,16 @@ def _load():
     lib.orc_taylor_coefficients.argtypes = [P]
     lib.orc_group_weight.argtypes = [f32, f32]
     lib.orc_group_weight.restype = u32
-    lib.orc_select_sample_group.argtypes = [P, P, i32, i32, ctypes.POINTER(_SelectCfg),
+    lib.orc_select_sample_group.argtypes = [P, P, i32, i32, ctypes.POINTER(_SelectCfg), P,
                                             P, P, P, P, P, P]
     lib.orc_select_sample_group.restype = i32
-    lib.orc_select_sample.argtypes = [P, i32, P, i32, i32, f32, P, ctypes.POINTER(_SelectCfg),
+    lib.orc_select_sample.argtypes = [P, i32, P, i32, i32, f32, P, ctypes.POINTER(_SelectCfg), P,
                                       P, P, P, P]
+    lib.orc_pq_codebook.argtypes = [P, i32, i32, P, P]
+    lib.orc_pq_codebook.restype = i32
+    lib.orc_pq_encode.argtypes = [P, i64, i32, P, i32, P]
+    lib.orc_pq_votes.argtypes = [P, i64, i32, P, P, i32, P, i32, P, i32, P, P, i32, i64, P]
+    lib.orc_pq_votes.restype = i32
     lib.orc_select_sample.restype = i32
     lib.orc_attention_rows.argtypes = [P, P, P, i64, i32, f32, P, P, P, i32, P, P, P, P, i64,
                                        P, i64, P]
@@ -206,10 +211,12 @@ def _cfg(E, m, seed, layer, bh, mode):
     return _SelectCfg(int(E), int(m), int(seed) & 0xFFFFFFFFFFFFFFFF, int(layer), int(bh), int(mode))
 
 
-def select_sample_group(S_row, k_offsets, i, E, m, seed=0, layer=0, bh=0, mode=IMPORTANCE):
+def select_sample_group(S_row, k_offsets, i, E, m, seed=0, layer=0, bh=0, mode=IMPORTANCE, votes=None):
     """One query group: dict with exact groups, counts, sample positions and
-    log-weights, the integer weights q_j (0 off the skipped set) and T."""
+    log-weights, the integer weights q_j (0 off the skipped set) and T.
+    ``votes`` ([Ck] int32): rank the exact set by votes first (PQ voting)."""
     lib = _load()
+    vrow = None if votes is None else _i32(votes)
     S_row = _f32(S_row)
     koff = _i32(k_offsets)
     Ck = S_row.shape[0]
@@ -220,7 +227,8 @@ def select_sample_group(S_row, k_offsets, i, E, m, seed=0, layer=0, bh=0, mode=I
     qw = np.zeros(Ck, np.uint32)
     tot = ctypes.c_uint64(0)
     cfg = _cfg(E, m, seed, layer, bh, mode)
-    _check(lib.orc_select_sample_group(_ptr(S_row), _ptr(koff), Ck, i, ctypes.byref(cfg), _ptr(ex),
+    _check(lib.orc_select_sample_group(_ptr(S_row), _ptr(koff), Ck, i, ctypes.byref(cfg),
+                                       None if vrow is None else _ptr(vrow), _ptr(ex),
                                        _ptr(cnt), _ptr(pos), _ptr(bias), _ptr(qw), ctypes.byref(tot)),
            "select_sample_group")
     ne, _, ns = (int(v) for v in cnt)
@@ -228,10 +236,11 @@ def select_sample_group(S_row, k_offsets, i, E, m, seed=0, layer=0, bh=0, mode=I
                 sample_pos=pos[:ns].copy(), sample_bias=bias[:ns].copy(), q=qw, total=int(tot.value))
 
 
-def select_sample(cq, ck, k_offsets, scale, E, m, seed=0, layer=0, bh=0, mode=IMPORTANCE):
+def select_sample(cq, ck, k_offsets, scale, E, m, seed=0, layer=0, bh=0, mode=IMPORTANCE, votes=None):
     """Whole head: (exact_groups [Cq,Ck], counts [Cq,3], sample_pos [Cq,m],
-    sample_bias [Cq,m] fp64)."""
+    sample_bias [Cq,m] fp64).  ``votes`` [Cq,Ck]: PQ-voting ranking."""
     lib = _load()
+    vv = None if votes is None else _i32(votes)
     cq, ck, koff = _f32(cq), _f32(ck), _i32(k_offsets)
     Cq, d = cq.shape
     Ck = ck.shape[0]
@@ -241,9 +250,57 @@ def select_sample(cq, ck, k_offsets, scale, E, m, seed=0, layer=0, bh=0, mode=IM
     bias = np.empty((Cq, max(m, 1)), np.float64)
     cfg = _cfg(E, m, seed, layer, bh, mode)
     _check(lib.orc_select_sample(_ptr(cq), Cq, _ptr(ck), Ck, d, float(np.float32(scale)), _ptr(koff),
-                                 ctypes.byref(cfg), _ptr(ex), _ptr(cnt), _ptr(pos), _ptr(bias)),
+                                 ctypes.byref(cfg), None if vv is None else _ptr(vv), _ptr(ex), _ptr(cnt),
+                                 _ptr(pos), _ptr(bias)),
            "select_sample")
     return ex, cnt, pos[:, :m], bias[:, :m]
+
+
+# ------------------------------------------------------------ PQ voting (readings
+# in the C source: 8-dimension subspaces, 16 codewords, 5 Lloyd iterations on
+# the group centroids, per-query budget prefix, votes then centroid score)
+PQ_SUB, PQ_KC, PQ_ITERS = 8, 16, 5
+
+
+def pq_codebook(P):
+    """Codebook of the points P [C,d]: (cb [M,16,8] fp32, codes [C,M] uint8,
+    codewords in use)."""
+    lib = _load()
+    P = _f32(P)
+    C, d = P.shape
+    M = d // PQ_SUB
+    cb = np.zeros((M, PQ_KC, PQ_SUB), np.float32)
+    codes = np.zeros((C, M), np.uint8)
+    kc = lib.orc_pq_codebook(_ptr(P), C, d, _ptr(cb), _ptr(codes))
+    if kc < 1:
+        raise ValueError("pq_codebook: bad shape")
+    return cb, codes, int(kc)
+
+
+def pq_encode(X, cb, kc):
+    """codes [n,M] of the rows X [n,d] against cb (kc codewords in use)."""
+    lib = _load()
+    X = _f32(X)
+    n, d = X.shape
+    codes = np.zeros((n, d // PQ_SUB), np.uint8)
+    lib.orc_pq_encode(_ptr(X), n, d, _ptr(np.ascontiguousarray(cb, np.float32)), int(kc), _ptr(codes))
+    return codes
+
+
+def pq_votes(Q, cq, ck, q_perm, q_offsets, k_offsets, E):
+    """Votes [Cq,Ck] of one head: codebooks from the centroids, key groups
+    encoded by their centroids, each query voting for its budget prefix."""
+    lib = _load()
+    Q = _f32(Q)
+    N, d = Q.shape
+    cbq, _, kcq = pq_codebook(cq)
+    cbk, kcodes, kck = pq_codebook(ck)
+    qp, qo, ko = _i32(q_perm), _i32(q_offsets), _i32(k_offsets)
+    Cq, Ck = qo.shape[0] - 1, ko.shape[0] - 1
+    votes = np.zeros((Cq, Ck), np.int32)
+    _check(lib.orc_pq_votes(_ptr(Q), N, d, _ptr(qp), _ptr(qo), Cq, _ptr(cbq), kcq, _ptr(cbk), kck,
+                            _ptr(np.ascontiguousarray(kcodes)), _ptr(ko), Ck, int(E), _ptr(votes)), "pq_votes")
+    return votes
 
 
 # ---------------------------------------------------------------------- attention
@@ -287,9 +344,11 @@ class HeadResult:
 
 
 def forward_head(Q, K, V, *, Cq, Ck, iters, exact_frac, sample_frac, scale, seed=0, layer=0, bh=0,
-                 mode=IMPORTANCE, rows=None, cq_init=None, ck_init=None) -> HeadResult:
+                 mode=IMPORTANCE, rows=None, cq_init=None, ck_init=None, selection="centroid") -> HeadResult:
     """All stages for one head, in the pages' order.  ``rows`` limits the
-    attention stage to those original query indices (all when None)."""
+    attention stage to those original query indices (all when None).
+    ``selection``: "centroid" (Figure 3) or "pq_vote" (the abstract's
+    product-quantised per-query voting)."""
     Q, K, V = _f32(Q), _f32(K), _f32(V)
     N = Q.shape[0]
     cq, qa, _ = kmeans(Q, Cq, iters, cq_init)
@@ -297,7 +356,8 @@ def forward_head(Q, K, V, *, Cq, Ck, iters, exact_frac, sample_frac, scale, seed
     qp, qo = permutation(qa, Cq)
     kp, ko = permutation(ka, Ck)
     E, m = budget(exact_frac, N), budget(sample_frac, N)
-    ex, cnt, sp, sb = select_sample(cq, ck, ko, scale, E, m, seed, layer, bh, mode)
+    votes = pq_votes(Q, cq, ck, qp, qo, ko, E) if selection == "pq_vote" else None
+    ex, cnt, sp, sb = select_sample(cq, ck, ko, scale, E, m, seed, layer, bh, mode, votes)
     if rows is None:
         rows = np.arange(N)
     out = attention_rows(Q, K, V, scale, qa, kp, ko, ex, cnt, sp, sb, rows) if len(rows) else None

@@ -298,7 +298,7 @@ typedef struct {
 } orc_select_cfg;
 
 int orc_select_sample_group(const float* S_row, const int32_t* k_offsets, int Ck, int i,
-                            const orc_select_cfg* cfg,
+                            const orc_select_cfg* cfg, const int32_t* votes_row /* [Ck] or NULL */,
                             int32_t* exact_groups, int32_t* counts,
                             int32_t* sample_pos, double* sample_bias,
                             uint32_t* qw_out /* [Ck] or NULL: 0 for non-skipped */,
@@ -310,7 +310,8 @@ int orc_select_sample_group(const float* S_row, const int32_t* k_offsets, int Ck
     uint64_t* cdf = (uint64_t*)calloc((size_t)(Ck > 0 ? Ck : 1), sizeof(uint64_t));
     if (!order || !in_exact || !qw || !cdf) { free(order); free(in_exact); free(qw); free(cdf); return ORC_ERR_NOMEM; }
 
-    /* rank the non-empty groups: plain insertion sort, S descending, j ascending */
+    /* rank the non-empty groups: plain insertion sort, S descending, j
+     * ascending; with votes (product-quantised voting), votes descending first */
     int nz = 0;
     for (int j = 0; j < Ck; ++j) {
         if (k_offsets[j + 1] - k_offsets[j] <= 0) continue;
@@ -319,6 +320,7 @@ int orc_select_sample_group(const float* S_row, const int32_t* k_offsets, int Ck
             int prev = order[pos - 1];
             float sp = S_row[prev], sj = S_row[j];
             int before = (sp > sj) || (sp == sj && prev < j);
+            if (votes_row && votes_row[prev] != votes_row[j]) before = votes_row[prev] > votes_row[j];
             if (before) break;
             order[pos] = prev;
             --pos;
@@ -391,6 +393,7 @@ int orc_select_sample_group(const float* S_row, const int32_t* k_offsets, int Ck
  * Unused sample slots hold position -1 and log-weight 0.                      */
 int orc_select_sample(const float* cq, int Cq, const float* ck, int Ck, int d, float scale,
                       const int32_t* k_offsets, const orc_select_cfg* cfg,
+                      const int32_t* votes /* [Cq][Ck] or NULL */,
                       int32_t* exact_groups, int32_t* counts,
                       int32_t* sample_pos, double* sample_bias)
 {
@@ -403,10 +406,170 @@ int orc_select_sample(const float* cq, int Cq, const float* ck, int Ck, int d, f
         double* sb = sample_bias + (int64_t)i * cfg->m;
         for (int64_t t = 0; t < cfg->m; ++t) { sp[t] = -1; sb[t] = 0.0; }
         rc = orc_select_sample_group(S + (int64_t)i * Ck, k_offsets, Ck, i, cfg,
+                                     votes ? votes + (int64_t)i * Ck : NULL,
                                      exact_groups + (int64_t)i * Ck, counts + 3 * i,
                                      sp, sb, NULL, NULL);
     }
     free(S);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Product-quantised per-query voting (the selection rule of the abstract:
+ * queries and keys are product-quantised so that a block score is cheap for
+ * every query, each query votes for its top blocks, and the cluster attends
+ * to the most-voted blocks).  The pages fix nothing beyond that sentence;
+ * every parameter below is a [reading]:
+ *   - subspaces of 8 consecutive dimensions (M = d/8), 16 codewords each, one
+ *     codebook per side (queries, keys) and head;
+ *   - a codebook is trained by 5 Lloyd iterations on the group centroids of
+ *     its side (cq for queries, ck for keys), initialised with the first
+ *     min(16, C) of them; distances sum (x_e - c_e)^2 with fmaf over e = 0..7
+ *     from +0; ties go to the lowest codeword; a codeword's update is the
+ *     fp32 sum of its members in point order divided by their count (fp32);
+ *     an empty codeword keeps its value;
+ *   - a query token is encoded against the query codebook, a key group by
+ *     its centroid against the key codebook (nearest codeword, same rule);
+ *   - block score s(q, j) = sum over m = 0..M-1 (fp32 adds from +0) of
+ *     T_m[a_m(q)][b_m(j)], T_m[a][b] = the fmaf chain over e of the two
+ *     codewords' products;
+ *   - query q votes for the prefix of its ranking (non-empty groups by s
+ *     descending, ties lowest j) chosen by the exact-set budget rule: rank 0
+ *     always, then while the running key count stays <= E;
+ *   - the group ranks key groups by votes descending, then by the centroid
+ *     score S_ij descending and j ascending, and takes the exact set by the
+ *     same budget rule; pi and the sample stay those of the centroid scores.
+ * Every decision is a correctly rounded fp32 operation in a fixed order, so
+ * an implementation that follows the same order agrees bit for bit.          */
+/* ------------------------------------------------------------------------- */
+#define ORC_PQ_SUB 8
+#define ORC_PQ_KC 16
+#define ORC_PQ_ITERS 5
+
+static float orc_pq_dist(const float* x, const float* c)
+{
+    float acc = 0.0f;
+    for (int e = 0; e < ORC_PQ_SUB; ++e) {
+        float t = x[e] - c[e];
+        acc = fmaf(t, t, acc);
+    }
+    return acc;
+}
+
+/* nearest of kc codewords (cb: kc x 8), ties to the lowest index */
+static int orc_pq_nearest(const float* x, const float* cb, int kc)
+{
+    int best = 0;
+    float bd = orc_pq_dist(x, cb);
+    for (int c = 1; c < kc; ++c) {
+        float dd = orc_pq_dist(x, cb + (size_t)c * ORC_PQ_SUB);
+        if (dd < bd) { bd = dd; best = c; }
+    }
+    return best;
+}
+
+/* Codebook of C points P [C, d] (d % 8 == 0): cb [M][16][8] (codewords past
+ * min(16, C) are zero and never chosen), codes [C][M] of the points against
+ * the final codebook.  Returns the number of codewords in use.               */
+int orc_pq_codebook(const float* P, int C, int d, float* cb, uint8_t* codes)
+{
+    const int M = d / ORC_PQ_SUB;
+    const int kc = C < ORC_PQ_KC ? C : ORC_PQ_KC;
+    if (C < 1 || d % ORC_PQ_SUB) return -1;
+    memset(cb, 0, sizeof(float) * (size_t)M * ORC_PQ_KC * ORC_PQ_SUB);
+    int* a = (int*)malloc(sizeof(int) * (size_t)C);
+    if (!a) return -1;
+    for (int m = 0; m < M; ++m) {
+        float* cbm = cb + (size_t)m * ORC_PQ_KC * ORC_PQ_SUB;
+        for (int c = 0; c < kc; ++c)
+            for (int e = 0; e < ORC_PQ_SUB; ++e) cbm[c * ORC_PQ_SUB + e] = P[(size_t)c * d + m * ORC_PQ_SUB + e];
+        for (int it = 0; it < ORC_PQ_ITERS; ++it) {
+            for (int p = 0; p < C; ++p) a[p] = orc_pq_nearest(P + (size_t)p * d + m * ORC_PQ_SUB, cbm, kc);
+            for (int c = 0; c < kc; ++c) {
+                float sum[ORC_PQ_SUB] = {0};
+                int n = 0;
+                for (int p = 0; p < C; ++p) {
+                    if (a[p] != c) continue;
+                    for (int e = 0; e < ORC_PQ_SUB; ++e) sum[e] += P[(size_t)p * d + m * ORC_PQ_SUB + e];
+                    ++n;
+                }
+                if (n > 0)
+                    for (int e = 0; e < ORC_PQ_SUB; ++e) cbm[c * ORC_PQ_SUB + e] = sum[e] / (float)n;
+            }
+        }
+        if (codes)
+            for (int p = 0; p < C; ++p)
+                codes[(size_t)p * M + m] = (uint8_t)orc_pq_nearest(P + (size_t)p * d + m * ORC_PQ_SUB, cbm, kc);
+    }
+    free(a);
+    return kc;
+}
+
+/* codes [n][M] of the rows X [n, d] against cb (kc codewords in use) */
+void orc_pq_encode(const float* X, int64_t n, int d, const float* cb, int kc, uint8_t* codes)
+{
+    const int M = d / ORC_PQ_SUB;
+    for (int64_t p = 0; p < n; ++p)
+        for (int m = 0; m < M; ++m)
+            codes[p * M + m] = (uint8_t)orc_pq_nearest(X + p * d + m * ORC_PQ_SUB,
+                                                       cb + (size_t)m * ORC_PQ_KC * ORC_PQ_SUB, kc);
+}
+
+/* Votes of one head: Q [N, d] (original token order), query groups through
+ * q_perm / q_offsets, the two codebooks (kcq, kck codewords in use), the key
+ * groups' codes kcodes [Ck][M] and k_offsets; votes [Cq][Ck].                */
+int orc_pq_votes(const float* Q, int64_t N, int d, const int32_t* q_perm, const int32_t* q_offsets, int Cq,
+                 const float* cbq, int kcq, const float* cbk, int kck, const uint8_t* kcodes,
+                 const int32_t* k_offsets, int Ck, int64_t E, int32_t* votes)
+{
+    const int M = d / ORC_PQ_SUB;
+    float* T = (float*)malloc(sizeof(float) * (size_t)M * ORC_PQ_KC * ORC_PQ_KC);
+    float* s = (float*)malloc(sizeof(float) * (size_t)(Ck > 0 ? Ck : 1));
+    int32_t* order = (int32_t*)malloc(sizeof(int32_t) * (size_t)(Ck > 0 ? Ck : 1));
+    uint8_t* qc = (uint8_t*)malloc((size_t)M);
+    if (!T || !s || !order || !qc) { free(T); free(s); free(order); free(qc); return ORC_ERR_NOMEM; }
+    for (int m = 0; m < M; ++m)
+        for (int a = 0; a < ORC_PQ_KC; ++a)
+            for (int b = 0; b < ORC_PQ_KC; ++b) {
+                const float* x = cbq + ((size_t)m * ORC_PQ_KC + a) * ORC_PQ_SUB;
+                const float* y = cbk + ((size_t)m * ORC_PQ_KC + b) * ORC_PQ_SUB;
+                float acc = 0.0f;
+                for (int e = 0; e < ORC_PQ_SUB; ++e) acc = fmaf(x[e], y[e], acc);
+                T[((size_t)m * ORC_PQ_KC + a) * ORC_PQ_KC + b] = acc;
+            }
+    memset(votes, 0, sizeof(int32_t) * (size_t)Cq * (size_t)Ck);
+    int rc = ORC_OK;
+    for (int i = 0; i < Cq && rc == ORC_OK; ++i) {
+        for (int64_t slot = q_offsets[i]; slot < q_offsets[i + 1]; ++slot) {
+            const int64_t q = q_perm[slot];
+            if (q < 0 || q >= N) { rc = ORC_ERR_ARG; break; }
+            orc_pq_encode(Q + q * d, 1, d, cbq, kcq, qc);
+            int nz = 0;
+            for (int j = 0; j < Ck; ++j) {
+                if (k_offsets[j + 1] - k_offsets[j] <= 0) continue;
+                float acc = 0.0f;
+                for (int m = 0; m < M; ++m)
+                    acc += T[((size_t)m * ORC_PQ_KC + qc[m]) * ORC_PQ_KC + kcodes[(size_t)j * M + m]];
+                s[j] = acc;
+                int pos = nz++;  /* insertion sort: s descending, j ascending */
+                while (pos > 0 && !(s[order[pos - 1]] > acc || (s[order[pos - 1]] == acc && order[pos - 1] < j))) {
+                    order[pos] = order[pos - 1];
+                    --pos;
+                }
+                order[pos] = j;
+            }
+            int64_t keys = 0;
+            for (int r = 0; r < nz; ++r) {
+                const int j = order[r];
+                const int64_t cnt = k_offsets[j + 1] - k_offsets[j];
+                if (r > 0 && keys + cnt > E) break;
+                keys += cnt;
+                votes[(int64_t)i * Ck + j] += 1;
+            }
+        }
+    }
+    (void)kck;
+    free(T); free(s); free(order); free(qc);
     return rc;
 }
 
