@@ -25,6 +25,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "_build", "libinstagen.so")
 
 IMPORTANCE, UNIFORM = 0, 1
+CENTROID, PQ_VOTE = 0, 1  # instagen_selection
 
 
 class InstaGenError(RuntimeError):
@@ -37,14 +38,14 @@ class Params(ctypes.Structure):
                 ("Cq", ctypes.c_int32), ("Ck", ctypes.c_int32), ("kmeans_iters", ctypes.c_int32),
                 ("exact_frac", ctypes.c_float), ("sample_frac", ctypes.c_float),
                 ("softmax_scale", ctypes.c_float), ("seed", ctypes.c_uint64), ("layer", ctypes.c_uint32),
-                ("sampling", ctypes.c_int32)]
+                ("sampling", ctypes.c_int32), ("selection", ctypes.c_int32)]
 
 
 class ForwardLayout(ctypes.Structure):
     """Mirror of ``instagen_forward_layout`` (byte offsets into the workspace)."""
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "cq", "ck", "q_assign", "k_assign", "q_perm", "k_perm", "q_offsets", "k_offsets", "kp", "vp",
-        "exact_groups", "counts", "sample_pos", "sample_bias", "cluster_ws", "total")]
+        "exact_groups", "counts", "sample_pos", "sample_bias", "votes", "pq_ws", "cluster_ws", "total")]
 
 
 _lib = None
@@ -53,7 +54,8 @@ _SYMBOLS = ("instagen_exact_budget", "instagen_sample_budget", "instagen_workspa
             "instagen_cluster", "instagen_permutation", "instagen_gather", "instagen_select_sample",
             "instagen_attention", "instagen_forward", "instagen_forward_layout_get",
             "instagen_cluster_static", "instagen_forward_host_workspace_size", "instagen_forward_host",
-            "instagen_forward_init")
+            "instagen_forward_init", "instagen_pq_votes_workspace_size", "instagen_pq_votes",
+            "instagen_select_sample_votes")
 
 
 def lib():
@@ -84,6 +86,9 @@ def lib():
         "instagen_forward_host_workspace_size": (sz, [P, i32]),
         "instagen_forward_host": (ctypes.c_int, [PP, PP, PP, PP, P, i32, PP, sz, vp]),
         "instagen_forward_init": (ctypes.c_int, [PP, PP, PP, PP, P, PP, PP, PP, sz, vp]),
+        "instagen_pq_votes_workspace_size": (sz, [P]),
+        "instagen_pq_votes": (ctypes.c_int, [PP, PP, PP, PP, PP, PP, P, PP, PP, sz, vp]),
+        "instagen_select_sample_votes": (ctypes.c_int, [PP, PP, PP, PP, P, PP, PP, PP, PP, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -122,11 +127,14 @@ def _need(t: torch.Tensor, name: str, dtype, shape=None):
 
 def make_params(B: int, H: int, N: int, d: int, Cq: int, Ck: int, *, iters: int = 10, exact_frac: float = 0.16,
                 sample_frac: float = 0.16, softmax_scale: Optional[float] = None, seed: int = 0, layer: int = 0,
-                sampling: int | str = IMPORTANCE) -> Params:
+                sampling: int | str = IMPORTANCE, selection: int | str = CENTROID) -> Params:
     if isinstance(sampling, str):
         sampling = {"importance": IMPORTANCE, "uniform": UNIFORM}[sampling]
+    if isinstance(selection, str):
+        selection = {"centroid": CENTROID, "pq_vote": PQ_VOTE}[selection]
     scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
-    return Params(B, H, N, d, Cq, Ck, iters, exact_frac, sample_frac, scale, seed & (2 ** 64 - 1), layer, sampling)
+    return Params(B, H, N, d, Cq, Ck, iters, exact_frac, sample_frac, scale, seed & (2 ** 64 - 1), layer, sampling,
+                  selection)
 
 
 def exact_budget(p: Params) -> int:
@@ -222,9 +230,29 @@ def gather(X: torch.Tensor, perm: torch.Tensor, p: Params, to_f16: bool = False)
     return Xp
 
 
-def select_sample(cq: torch.Tensor, ck: torch.Tensor, k_offsets: torch.Tensor, p: Params):
+def pq_votes(Q: torch.Tensor, cq: torch.Tensor, ck: torch.Tensor, q_perm: torch.Tensor, q_offsets: torch.Tensor,
+             k_offsets: torch.Tensor, p: Params) -> torch.Tensor:
+    """Product-quantised per-query votes [B,H,Cq,Ck] int32 (instagen_pq_votes)."""
+    _need(Q, "Q", torch.bfloat16, (p.B, p.H, p.N, p.d))
+    _need(cq, "cq", torch.float32, (p.B, p.H, p.Cq, p.d))
+    _need(ck, "ck", torch.float32, (p.B, p.H, p.Ck, p.d))
+    _need(q_perm, "q_perm", torch.int32, (p.B, p.H, p.N))
+    _need(q_offsets, "q_offsets", torch.int32, (p.B, p.H, p.Cq + 1))
+    _need(k_offsets, "k_offsets", torch.int32, (p.B, p.H, p.Ck + 1))
+    votes = torch.empty((p.B, p.H, p.Cq, p.Ck), dtype=torch.int32, device=Q.device)
+    nws = int(lib().instagen_pq_votes_workspace_size(ctypes.byref(p)))
+    ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=Q.device)
+    _check(lib().instagen_pq_votes(_ptr(Q), _ptr(cq), _ptr(ck), _ptr(q_perm), _ptr(q_offsets), _ptr(k_offsets),
+                                   ctypes.byref(p), _ptr(votes), _ptr(ws), ws.numel(), _stream()),
+           "instagen_pq_votes")
+    return votes
+
+
+def select_sample(cq: torch.Tensor, ck: torch.Tensor, k_offsets: torch.Tensor, p: Params,
+                  votes: Optional[torch.Tensor] = None):
     """Returns (exact_groups [B,H,Cq,Ck], counts [B,H,Cq,3], sample_pos [B,H,Cq,m] int32,
-    sample_bias [B,H,Cq,m] fp32)."""
+    sample_bias [B,H,Cq,m] fp32).  With ``votes`` [B,H,Cq,Ck] int32 the exact
+    set is ranked by votes first (instagen_select_sample_votes)."""
     _need(cq, "cq", torch.float32, (p.B, p.H, p.Cq, p.d))
     _need(ck, "ck", torch.float32, (p.B, p.H, p.Ck, p.d))
     _need(k_offsets, "k_offsets", torch.int32, (p.B, p.H, p.Ck + 1))
@@ -234,6 +262,13 @@ def select_sample(cq: torch.Tensor, ck: torch.Tensor, k_offsets: torch.Tensor, p
     cnt = torch.empty((p.B, p.H, p.Cq, 3), dtype=torch.int32, device=dev)
     sp = torch.empty((p.B, p.H, p.Cq, m), dtype=torch.int32, device=dev)
     sb = torch.empty((p.B, p.H, p.Cq, m), dtype=torch.float32, device=dev)
+    if votes is not None:
+        _need(votes, "votes", torch.int32, (p.B, p.H, p.Cq, p.Ck))
+        _check(lib().instagen_select_sample_votes(_ptr(cq), _ptr(ck), _ptr(k_offsets), _ptr(votes), ctypes.byref(p),
+                                                  _ptr(eg), _ptr(cnt), _ptr(sp) if m else None,
+                                                  _ptr(sb) if m else None, _stream()),
+               "instagen_select_sample_votes")
+        return eg, cnt, sp, sb
     _check(lib().instagen_select_sample(_ptr(cq), _ptr(ck), _ptr(k_offsets), ctypes.byref(p), _ptr(eg), _ptr(cnt),
                                         _ptr(sp) if m else None, _ptr(sb) if m else None, _stream()),
            "instagen_select_sample")
@@ -347,4 +382,5 @@ def forward_intermediates(workspace: torch.Tensor, p: Params) -> dict:
         counts=view(L.counts, B * H * Cq * 3, torch.int32, (B, H, Cq, 3)),
         sample_pos=view(L.sample_pos, B * H * Cq * m, torch.int32, (B, H, Cq, m)),
         sample_bias=view(L.sample_bias, B * H * Cq * m, torch.float32, (B, H, Cq, m)),
+        **({"votes": view(L.votes, B * H * Cq * Ck, torch.int32, (B, H, Cq, Ck))} if p.selection == PQ_VOTE else {}),
     )

@@ -36,6 +36,9 @@ int check_params(const instagen_params* p) {
     return IG_ERR_INVALID_ARG;
   if (!std::isfinite(p->softmax_scale) || !(p->softmax_scale > 0.f)) return IG_ERR_INVALID_ARG;
   if (p->sampling != IG_SAMPLE_IMPORTANCE && p->sampling != IG_SAMPLE_UNIFORM) return IG_ERR_INVALID_ARG;
+  if (p->selection != IG_SELECT_CENTROID && p->selection != IG_SELECT_PQ_VOTE) return IG_ERR_INVALID_ARG;
+  // votes enter the rank key saturated at 2^20 - 1: a group has fewer queries
+  if (p->selection == IG_SELECT_PQ_VOTE && p->N > 0xFFFFF) return IG_ERR_UNSUPPORTED;
   return IG_OK;
 }
 
@@ -144,6 +147,9 @@ int forward_layout(const instagen_params* p, instagen_forward_layout* L) {
   L->counts = take(BH * p->Cq * 3 * 4);
   L->sample_pos = take(BH * p->Cq * (m ? m : 1) * 4);
   L->sample_bias = take(BH * p->Cq * (m ? m : 1) * 4);
+  const bool pq = p->selection == IG_SELECT_PQ_VOTE;
+  L->votes = take(pq ? BH * p->Cq * p->Ck * 4 : 0);
+  L->pq_ws = take(pq ? ig::pq_scratch_bytes((int)BH, p->d, p->Ck) : 0);
   const size_t cq_ws = ig::kmeans_scratch_bytes(ig::kmeans_geom((int)BH, p->N, p->d, p->Cq));
   const size_t ck_ws = ig::kmeans_scratch_bytes(ig::kmeans_geom((int)BH, p->N, p->d, p->Ck));
   L->cluster_ws = take(cq_ws > ck_ws ? cq_ws : ck_ws);
@@ -154,7 +160,7 @@ int forward_layout(const instagen_params* p, instagen_forward_layout* L) {
 // bh0: global index of the first head (the sample's Philox counter uses it).
 int select_impl(const float* cq, const float* ck, const int32_t* k_offsets, const instagen_params* p,
                 int32_t* exact_groups, int32_t* counts, int32_t* sample_pos, float* sample_bias, int bh0,
-                void* stream) {
+                void* stream, const int32_t* votes = nullptr) {
   int rc = check_params(p);
   if (rc) return rc;
   if ((rc = check_clusters(p->Cq)) || (rc = check_clusters(p->Ck))) return rc;
@@ -177,6 +183,7 @@ int select_impl(const float* cq, const float* ck, const int32_t* k_offsets, cons
   a.layer = p->layer;
   a.mode = p->sampling;
   a.bh0 = bh0;
+  a.votes = votes;
   a.exact_groups = exact_groups;
   a.counts = counts;
   a.sample_pos = sample_pos;
@@ -222,7 +229,13 @@ int forward_impl(const void* Q, const void* K, const void* V, void* O, const ins
   rc = cuda_status(ig::launch_gather_rows(static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V),
                                           kp, p->B * p->H, p->N, p->d, Kp, Vp, false, true, s));
   if (rc) return rc;
-  rc = select_impl(cq, ck, ko, p, eg, cnt, sp, sb, bh0, stream);
+  int32_t* votes = nullptr;
+  if (p->selection == IG_SELECT_PQ_VOTE) {
+    votes = reinterpret_cast<int32_t*>(w + L.votes);
+    rc = instagen_pq_votes(Q, cq, ck, qp, qo, ko, p, votes, w + L.pq_ws, L.cluster_ws - L.pq_ws, stream);
+    if (rc) return rc;
+  }
+  rc = select_impl(cq, ck, ko, p, eg, cnt, sp, sb, bh0, stream, votes);
   if (rc) return rc;
   return instagen_attention(Q, Kp, Vp, qp, qo, ko, eg, cnt, sp, sb, p, O, stream);
 }
@@ -338,6 +351,49 @@ int instagen_gather(const void* X, const int32_t* perm, const instagen_params* p
   return cuda_status(ig::launch_gather_rows(static_cast<const __nv_bfloat16*>(X), nullptr, perm, p->B * p->H,
                                             p->N, p->d, Xp, nullptr, to_f16 != 0, false,
                                             static_cast<cudaStream_t>(stream)));
+}
+
+size_t instagen_pq_votes_workspace_size(const instagen_params* p) {
+  if (check_params(p) || check_clusters(p->Cq) || check_clusters(p->Ck)) return 0;
+  return ig::pq_scratch_bytes(p->B * p->H, p->d, p->Ck);
+}
+
+int instagen_pq_votes(const void* Q, const float* cq, const float* ck, const int32_t* q_perm,
+                      const int32_t* q_offsets, const int32_t* k_offsets, const instagen_params* p, int32_t* votes,
+                      void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if ((rc = check_clusters(p->Cq)) || (rc = check_clusters(p->Ck))) return rc;
+  if ((rc = check_budgets(p))) return rc;
+  if (p->N > 0xFFFFF) return IG_ERR_UNSUPPORTED;
+  if (!Q || !cq || !ck || !q_perm || !q_offsets || !k_offsets || !votes || !aligned16(Q)) return IG_ERR_INVALID_ARG;
+  const int BH = p->B * p->H;
+  if (!ws || ws_bytes < ig::pq_scratch_bytes(BH, p->d, p->Ck) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return IG_ERR_WORKSPACE;
+  ig::PqArgs a;
+  a.cq = cq;
+  a.ck = ck;
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
+  a.q_perm = q_perm;
+  a.q_offsets = q_offsets;
+  a.k_offsets = k_offsets;
+  a.BH = BH;
+  a.N = p->N;
+  a.d = p->d;
+  a.Cq = p->Cq;
+  a.Ck = p->Ck;
+  a.E = budget(p->exact_frac, p->N);
+  a.codebooks = nullptr;
+  a.kcodes = nullptr;
+  a.votes = votes;
+  return cuda_status(ig::launch_pq_votes(a, ws, static_cast<cudaStream_t>(stream)));
+}
+
+int instagen_select_sample_votes(const float* cq, const float* ck, const int32_t* k_offsets, const int32_t* votes,
+                                 const instagen_params* p, int32_t* exact_groups, int32_t* counts,
+                                 int32_t* sample_pos, float* sample_bias, void* stream) {
+  if (!votes) return IG_ERR_INVALID_ARG;
+  return select_impl(cq, ck, k_offsets, p, exact_groups, counts, sample_pos, sample_bias, 0, stream, votes);
 }
 
 int instagen_select_sample(const float* cq, const float* ck, const int32_t* k_offsets, const instagen_params* p,

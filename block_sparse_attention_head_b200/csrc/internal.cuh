@@ -61,12 +61,30 @@ struct SelectArgs {
   unsigned layer;
   int mode;
   int bh0;  // global index of head 0 of this launch (the Philox counter's head)
+  const int32_t* votes;  // [BH,Cq,Ck] product-quantised votes, or null (rank by S alone)
   int32_t* exact_groups;
   int32_t* counts;
   int32_t* sample_pos;
   float* sample_bias;
 };
 cudaError_t launch_select_sample(const SelectArgs& a, cudaStream_t s);
+
+// ------------------------------------------------- product-quantised votes
+struct PqArgs {
+  const float* cq;                  // [BH,Cq,d] query group centroids
+  const float* ck;                  // [BH,Ck,d] key group centroids
+  const __nv_bfloat16* Q;           // [BH,N,d] original order
+  const int32_t* q_perm;            // [BH,N]
+  const int32_t* q_offsets;         // [BH,Cq+1]
+  const int32_t* k_offsets;         // [BH,Ck+1]
+  int BH, N, d, Cq, Ck;
+  long long E;                      // exact-key budget
+  float* codebooks;                 // [BH][2][d/8][16][8] (set by launch_pq_votes)
+  uint8_t* kcodes;                  // [BH][Ck][d/8] (set by launch_pq_votes)
+  int32_t* votes;                   // [BH,Cq,Ck]
+};
+size_t pq_scratch_bytes(int BH, int d, int Ck);
+cudaError_t launch_pq_votes(const PqArgs& a, void* scratch, cudaStream_t s);
 
 // --------------------------------------------------------------- attention
 struct AttnArgs {

@@ -3,6 +3,7 @@
 #include "permute.cu"
 #include "kmeans.cu"
 #include "select.cu"
+#include "pqvote.cu"
 #include "attention.cu"
 #include "api.cu"
 #include "cluster_static.cu"

@@ -16,6 +16,7 @@ namespace ig {
 
 namespace {
 constexpr int kSelThreads = 512;
+constexpr unsigned long long kKeyJ = 0xFFFull;  // group index field of a rank key
 constexpr int kSelMaxCk = 4096;
 
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC 2011): ten rounds of two
@@ -148,11 +149,18 @@ __global__ void __launch_bounds__(kSelThreads)
   }
   __syncthreads();
 
-  // rank the non-empty groups: S descending, j ascending (bitonic sort of keys)
+  // rank the non-empty groups: S descending, j ascending (bitonic sort of
+  // keys; j < 4096 sits in the low 12 bits).  With votes (product-quantised
+  // voting) the votes, descending, come first (20 bits, saturated).
   for (int j = tid; j < ck_pow2; j += kSelThreads) {
     unsigned long long key = ~0ull;
-    if (j < Ck && koff[j + 1] > koff[j])
-      key = ((unsigned long long)(~float_order(S[j])) << 32) | (unsigned)j;
+    if (j < Ck && koff[j + 1] > koff[j]) {
+      key = ((unsigned long long)(~float_order(S[j])) << 12) | (unsigned)j;
+      if (a.votes) {
+        const int v = min(max(a.votes[gi * Ck + j], 0), 0xFFFFF);
+        key |= (unsigned long long)(0xFFFFF - v) << 44;
+      }
+    }
     keys[j] = key;
   }
   __syncthreads();
@@ -176,7 +184,7 @@ __global__ void __launch_bounds__(kSelThreads)
   // exact set: rank 0, then while the running key count stays <= E
   for (int r = tid; r < Ck; r += kSelThreads) {
     const unsigned long long key = keys[r];
-    cdf[r] = (key == ~0ull) ? 0ull : (unsigned long long)(koff[(key & 0xffffffffu) + 1] - koff[key & 0xffffffffu]);
+    cdf[r] = (key == ~0ull) ? 0ull : (unsigned long long)(koff[(key & kKeyJ) + 1] - koff[key & kKeyJ]);
   }
   __syncthreads();
   block_incl_scan_u64(cdf, Ck, wtot);  // cdf[r] = keys in ranks 0..r
@@ -191,11 +199,11 @@ __global__ void __launch_bounds__(kSelThreads)
   __syncthreads();
   const int n_exact = s_nexact;
   int32_t* ex_out = a.exact_groups + gi * Ck;
-  for (int r = tid; r < Ck; r += kSelThreads) ex_out[r] = r < n_exact ? (int32_t)(keys[r] & 0xffffffffu) : -1;
+  for (int r = tid; r < Ck; r += kSelThreads) ex_out[r] = r < n_exact ? (int32_t)(keys[r] & kKeyJ) : -1;
   // qw doubles as the exact-membership flag: 0 = exact or empty, 1 = skipped (for now)
   for (int j = tid; j < Ck; j += kSelThreads) qw[j] = (koff[j + 1] > koff[j]) ? 1u : 0u;
   __syncthreads();
-  for (int r = tid; r < n_exact; r += kSelThreads) qw[keys[r] & 0xffffffffu] = 0u;
+  for (int r = tid; r < n_exact; r += kSelThreads) qw[keys[r] & kKeyJ] = 0u;
   __syncthreads();
 
   // pi over the skipped groups

@@ -54,6 +54,10 @@ typedef enum {
 } instagen_status;
 
 typedef enum { IG_SAMPLE_IMPORTANCE = 0, IG_SAMPLE_UNIFORM = 1 } instagen_sampling;
+/* How the exact set is ranked: by centroid scores (Figure 3 (b)-(c)), or by
+ * product-quantised per-query votes (the abstract's rule; see
+ * instagen_pq_votes). */
+typedef enum { IG_SELECT_CENTROID = 0, IG_SELECT_PQ_VOTE = 1 } instagen_selection;
 
 typedef struct {
   int32_t B, H, N, d;        /* shapes; d in {64, 128}; N >= 1                     */
@@ -65,6 +69,7 @@ typedef struct {
   uint64_t seed;             /* Philox key                                           */
   uint32_t layer;            /* Philox counter word 3 (one stream per layer)         */
   int32_t sampling;          /* instagen_sampling                                    */
+  int32_t selection;         /* instagen_selection (PQ voting needs N < 2^20)        */
 } instagen_params;
 
 /* E and m for these parameters: the share times N rounded to nearest, halves
@@ -186,6 +191,40 @@ int instagen_gather(const void* X, const int32_t* perm, const instagen_params* p
  *   m = instagen_sample_budget(p); sample_pos/sample_bias may be NULL if m = 0.
  *   Requires Ck <= 4096.
  */
+/*
+ * Product-quantised per-query voting (abstract: queries and keys are product-
+ * quantised so a block score is cheap for every query, not only for the
+ * cluster centroid; each query votes for its top blocks; the cluster attends
+ * to the blocks with the most votes).  The pages fix nothing further; read
+ * here as: subspaces of 8 consecutive dimensions (M = d/8), 16 codewords per
+ * subspace and side, trained per head by 5 Lloyd iterations on that side's
+ * group centroids (start: the first min(16, C) centroids; squared distances
+ * as an fma chain of the 8 differences; ties to the lowest codeword; update
+ * = fp32 sum of the members in point order / their count; empty codewords
+ * keep their value); query tokens encoded against the query codebook, key
+ * groups by their centroids against the key codebook; block score = sum over
+ * m ascending (fp32 from +0) of T_m[a_m(q)][b_m(j)], T_m = fma-chain inner
+ * products of the two codebooks' codewords; query q votes for the prefix of
+ * its ranking (non-empty groups by score descending, ties lower j) that the
+ * exact-set budget rule takes (rank 0 always, then while the key count stays
+ * <= E).  Every decision is a correctly rounded fp32 step in a fixed order.
+ *   Q [B,H,N,d] bf16 original order; cq, ck, q_perm, q_offsets, k_offsets as
+ *   produced by instagen_cluster; votes [B,H,Cq,Ck] int32 (out).
+ *   ws: device scratch of instagen_pq_votes_workspace_size(p) bytes, 256-byte
+ *   aligned (codebooks and key-group codes).  Requires N < 2^20.
+ */
+size_t instagen_pq_votes_workspace_size(const instagen_params* p);
+int instagen_pq_votes(const void* Q, const float* cq, const float* ck, const int32_t* q_perm,
+                      const int32_t* q_offsets, const int32_t* k_offsets, const instagen_params* p, int32_t* votes,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* instagen_select_sample with the exact set ranked by votes [B,H,Cq,Ck]
+ * (descending; saturated at 2^20 - 1) before S_ij and j; pi and the sample
+ * as in instagen_select_sample. */
+int instagen_select_sample_votes(const float* cq, const float* ck, const int32_t* k_offsets, const int32_t* votes,
+                                 const instagen_params* p, int32_t* exact_groups, int32_t* counts,
+                                 int32_t* sample_pos, float* sample_bias, void* stream);
+
 int instagen_select_sample(const float* cq, const float* ck, const int32_t* k_offsets, const instagen_params* p,
                            int32_t* exact_groups, int32_t* counts, int32_t* sample_pos, float* sample_bias,
                            void* stream);
@@ -273,6 +312,8 @@ typedef struct {
   size_t kp, vp;                 /* [B,H,N,d] permuted K (bf16) and V (fp16)    */
   size_t exact_groups, counts;   /* int32 [B,H,Cq,Ck], [B,H,Cq,3]               */
   size_t sample_pos, sample_bias;/* int32 / fp32 [B,H,Cq,m]                     */
+  size_t votes, pq_ws;           /* PQ voting: int32 [B,H,Cq,Ck] and its scratch
+                                    (0 bytes unless selection = PQ voting)     */
   size_t cluster_ws;             /* scratch for instagen_cluster                */
   size_t total;                  /* == instagen_workspace_size                  */
 } instagen_forward_layout;

@@ -515,6 +515,18 @@ void orc_pq_encode(const float* X, int64_t n, int d, const float* cb, int kc, ui
                                                        cb + (size_t)m * ORC_PQ_KC * ORC_PQ_SUB, kc);
 }
 
+typedef struct { float s; int j; } orc_pq_ranked;
+
+/* ranking order: score descending, then the lower group index */
+static int orc_pq_rank_cmp(const void* pa, const void* pb)
+{
+    const orc_pq_ranked* a = (const orc_pq_ranked*)pa;
+    const orc_pq_ranked* b = (const orc_pq_ranked*)pb;
+    if (a->s > b->s) return -1;
+    if (a->s < b->s) return 1;
+    return (a->j > b->j) - (a->j < b->j);
+}
+
 /* Votes of one head: Q [N, d] (original token order), query groups through
  * q_perm / q_offsets, the two codebooks (kcq, kck codewords in use), the key
  * groups' codes kcodes [Ck][M] and k_offsets; votes [Cq][Ck].                */
@@ -524,10 +536,9 @@ int orc_pq_votes(const float* Q, int64_t N, int d, const int32_t* q_perm, const 
 {
     const int M = d / ORC_PQ_SUB;
     float* T = (float*)malloc(sizeof(float) * (size_t)M * ORC_PQ_KC * ORC_PQ_KC);
-    float* s = (float*)malloc(sizeof(float) * (size_t)(Ck > 0 ? Ck : 1));
-    int32_t* order = (int32_t*)malloc(sizeof(int32_t) * (size_t)(Ck > 0 ? Ck : 1));
+    orc_pq_ranked* order = (orc_pq_ranked*)malloc(sizeof(orc_pq_ranked) * (size_t)(Ck > 0 ? Ck : 1));
     uint8_t* qc = (uint8_t*)malloc((size_t)M);
-    if (!T || !s || !order || !qc) { free(T); free(s); free(order); free(qc); return ORC_ERR_NOMEM; }
+    if (!T || !order || !qc) { free(T); free(order); free(qc); return ORC_ERR_NOMEM; }
     for (int m = 0; m < M; ++m)
         for (int a = 0; a < ORC_PQ_KC; ++a)
             for (int b = 0; b < ORC_PQ_KC; ++b) {
@@ -550,17 +561,14 @@ int orc_pq_votes(const float* Q, int64_t N, int d, const int32_t* q_perm, const 
                 float acc = 0.0f;
                 for (int m = 0; m < M; ++m)
                     acc += T[((size_t)m * ORC_PQ_KC + qc[m]) * ORC_PQ_KC + kcodes[(size_t)j * M + m]];
-                s[j] = acc;
-                int pos = nz++;  /* insertion sort: s descending, j ascending */
-                while (pos > 0 && !(s[order[pos - 1]] > acc || (s[order[pos - 1]] == acc && order[pos - 1] < j))) {
-                    order[pos] = order[pos - 1];
-                    --pos;
-                }
-                order[pos] = j;
+                order[nz].s = acc;
+                order[nz].j = j;
+                ++nz;
             }
+            qsort(order, (size_t)nz, sizeof(orc_pq_ranked), orc_pq_rank_cmp);
             int64_t keys = 0;
             for (int r = 0; r < nz; ++r) {
-                const int j = order[r];
+                const int j = order[r].j;
                 const int64_t cnt = k_offsets[j + 1] - k_offsets[j];
                 if (r > 0 && keys + cnt > E) break;
                 keys += cnt;
@@ -569,7 +577,7 @@ int orc_pq_votes(const float* Q, int64_t N, int d, const int32_t* q_perm, const 
         }
     }
     (void)kck;
-    free(T); free(s); free(order); free(qc);
+    free(T); free(order); free(qc);
     return rc;
 }
 

@@ -34,10 +34,11 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_params_struct_layout():
-    # instagen_params: 7 int32, 3 float, uint64 (8-aligned at 40), uint32, int32
-    assert ctypes.sizeof(ig.Params) == 56
+    # instagen_params: 7 int32, 3 float, uint64 (8-aligned at 40), uint32, 2 int32
+    assert ctypes.sizeof(ig.Params) == 64
     assert ig.Params.seed.offset == 40
-    assert ctypes.sizeof(ig.ForwardLayout) == 16 * ctypes.sizeof(ctypes.c_size_t)
+    assert ig.Params.selection.offset == 56
+    assert ctypes.sizeof(ig.ForwardLayout) == 18 * ctypes.sizeof(ctypes.c_size_t)
 
 
 def test_budgets_match_oracle(lib, oracle_mod):
@@ -48,13 +49,19 @@ def test_budgets_match_oracle(lib, oracle_mod):
 
 
 def test_workspace_layout(lib):
-    p = ig.make_params(1, 40, 75600, 128, 100, 500)
+    # centroid selection: the PQ-voting blocks are empty
+    p0 = ig.make_params(1, 40, 75600, 128, 100, 500)
+    L0 = ig.forward_layout(p0)
+    assert L0.votes == L0.pq_ws == L0.cluster_ws
+    p = ig.make_params(1, 40, 75600, 128, 100, 500, selection="pq_vote")
     L = ig.forward_layout(p)
     fields = [f for f, _ in ig.ForwardLayout._fields_ if f != "total"]
     offs = [getattr(L, f) for f in fields]
     assert all(o % 256 == 0 for o in offs)
     assert offs == sorted(offs) and len(set(offs)) == len(offs)
     assert L.total == ig.workspace_size(p)
+    assert L.pq_ws - L.votes >= 40 * 100 * 500 * 4
+    assert L.total - L0.total == L.cluster_ws - L0.cluster_ws
     BH, N, d, m = 40, 75600, 128, 12096
     assert L.vp - L.kp >= BH * N * d * 2
     assert L.sample_bias - L.sample_pos >= BH * 100 * m * 4
@@ -117,3 +124,17 @@ def test_binding_refuses_cpu_tensors(lib):
     X = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16)
     with pytest.raises(ig.InstaGenError, match="CUDA tensor"):
         ig.forward(X, X, X, p)
+
+
+def test_pq_vote_selection_checks_on_host(lib):
+    """PQ voting keeps votes below 2^20 in the rank key: larger N is refused,
+    an unknown selection value is invalid, and the vote scratch is sized."""
+    p = ig.make_params(1, 1, 1 << 20, 64, 4, 8, selection="pq_vote")
+    assert lib.instagen_workspace_size(ctypes.byref(p)) == 0
+    p = ig.make_params(1, 1, (1 << 20) - 1, 64, 4, 8, selection="pq_vote")
+    assert lib.instagen_workspace_size(ctypes.byref(p)) > 0
+    p.selection = 7
+    assert lib.instagen_workspace_size(ctypes.byref(p)) == 0
+    p = ig.make_params(1, 40, 75600, 128, 100, 500, selection="pq_vote")
+    # codebooks [40][2][16][16][8] fp32 + key-group codes [40][500][16]
+    assert lib.instagen_pq_votes_workspace_size(ctypes.byref(p)) == 40 * 2 * 16 * 16 * 8 * 4 + 40 * 500 * 16
