@@ -44,6 +44,8 @@ def parse_args():
     ap.add_argument("--sample", type=float, default=None, help="override the sampled share")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the head count (same per-head shape; for profiling captures)")
+    ap.add_argument("--selection", default="centroid", choices=["centroid", "pq_vote"],
+                    help="exact-set ranking: centroid scores (default) or product-quantised per-query votes")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
@@ -202,9 +204,10 @@ def reference_arm(args, w, exact, sample):
     return 0
 
 
-def workload_config(w, exact, sample):
+def workload_config(w, exact, sample, selection="centroid"):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "Cq": w.Cq, "Ck": w.Ck,
             "kmeans_iters": w.iters, "exact_frac": exact, "sample_frac": sample, "sampling": "importance",
+            "selection": selection,
             "inputs": "clustered Gaussian mixture (seeded), bf16",
             "l2": "inputs (Q,K,V %.1f GB per call) larger than L2" % (3 * w.B * w.H * w.N * w.d * 2 / 1e9)}
 
@@ -246,7 +249,8 @@ def main():
     dev = torch.device("cuda", local)
     Q, K, V = workloads.make_inputs(w, layer=rank, device=dev)
     p = ig.make_params(w.B, w.H, w.N, w.d, w.Cq, w.Ck, iters=w.iters, exact_frac=exact, sample_frac=sample,
-                       seed=1000 + rank, layer=rank)
+                       seed=1000 + rank, layer=rank, selection=args.selection)
+    pq = args.selection == "pq_vote"
     ws = torch.empty(ig.workspace_size(p), dtype=torch.uint8, device=dev)
     O = torch.empty_like(Q)
     stream = torch.cuda.current_stream()
@@ -274,7 +278,7 @@ def main():
 
     # ---------------- stage breakdown: the same calls, staged, with events
     inter = ig.forward_intermediates(ws, p)
-    stages = ["cluster_q", "cluster_k", "gather_kv", "select_sample", "attention"]
+    stages = ["cluster_q", "cluster_k", "gather_kv"] + (["pq_votes"] if pq else []) + ["select_sample", "attention"]
     acc = {s: 0.0 for s in stages}
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
     barrier()
@@ -286,10 +290,14 @@ def main():
         evs[2].record(stream)
         Kp, Vp = ig.gather(K, kp, p), ig.gather(V, kp, p, to_f16=True)
         evs[3].record(stream)
-        eg, cnt, sp, sb = ig.select_sample(cq, ck, ko, p)
-        evs[4].record(stream)
+        votes = None
+        if pq:
+            votes = ig.pq_votes(Q, cq, ck, qp, qo, ko, p)
+            evs[4].record(stream)
+        eg, cnt, sp, sb = ig.select_sample(cq, ck, ko, p, votes=votes)
+        evs[len(stages) - 1].record(stream)
         ig.attention(Q, Kp, Vp, qp, qo, ko, eg, cnt, sp, sb, p, out=O)
-        evs[5].record(stream)
+        evs[len(stages)].record(stream)
         torch.cuda.synchronize()
         for i, s in enumerate(stages):
             acc[s] += evs[i].elapsed_time(evs[i + 1])
@@ -395,20 +403,20 @@ def main():
     value = ms_call / world
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not pq:  # the sample runs the centroid ranking
         orc = OracleSample(w, exact, sample)
         orc.step()
         vals = [orc.step() for _ in range(3)]
         cpu = {"value": round(statistics.median(vals), 1), "unit": "ms/call", "cores": orc.oracle.num_threads(),
                "kind": "oracle", "sample": orc.describe() + "; median of 3 steps"}
 
-    launches_per_step = 2 * (1 + 3 * w.iters) + 1 + 1 + 1
+    launches_per_step = 2 * (1 + 3 * w.iters) + 1 + 1 + 1 + (2 if pq else 0)  # + codebooks, votes
     peak_sust = peaks["bf16_sust"]
     line = {
         "metric": "ms per InstaGen attention call", "value": round(value, 3), "unit": "ms/call",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_call, 3),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(w, exact, sample),
+        "config": workload_config(w, exact, sample, args.selection),
         "effective_tflops": round(attended_flops / (ms_call * 1e-3) / 1e12, 1),
         "attended_flops": attended_flops, "density": round(density, 4),
         "roofline": {"kernel": "attention", "bound": "tensor", "achieved": round(achieved, 1),

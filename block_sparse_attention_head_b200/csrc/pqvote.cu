@@ -31,6 +31,7 @@ constexpr int kPqKc = 16;
 constexpr int kPqIters = 5;
 constexpr int kPqCbThreads = 128;
 constexpr int kPqVoteThreads = 256;
+constexpr int kPqChunk = 128;  // queries per CTA of the vote kernel
 
 __device__ __forceinline__ float pq_dist8(const float* x, const float* c) {
   float acc = 0.0f;
@@ -64,7 +65,7 @@ __device__ __forceinline__ int pq_nearest(const float* x, const float* cb, int k
 // groups' codes.
 __global__ void __launch_bounds__(kPqCbThreads)
     pq_codebook_kernel(PqArgs a) {
-  extern __shared__ uint8_t pq_sm[];
+  extern __shared__ __align__(16) uint8_t pq_sm[];
   uint8_t* asg = pq_sm;  // [C]
   __shared__ float cb[kPqKc * kPqSub];
   const int m = blockIdx.x, side = blockIdx.y, bh = blockIdx.z, tid = threadIdx.x;
@@ -125,25 +126,54 @@ __device__ __forceinline__ uint32_t pq_float_order(float s) {
 }
 }  // namespace
 
-// Votes of query group i of head bh: grid (Cq, BH), 8 warps, one query per
-// warp at a time.  A query's keys are ranked by the 44-bit key (score order
-// << 12 | 4095 - j): larger = earlier rank.  Its budget prefix is found by a
-// weighted radix select over that key (8, 8, 8, 8, 8 and 4 bits, weights =
-// key-group sizes): the select fixes, digit by digit, the key of the first
-// rank whose group no longer fits under E; the query votes for every key
-// above it (for the top key alone if even that one does not fit, for all if
-// every group fits).  Keys are distinct, so the prefix is exact.
+// Votes of a chunk of at most kPqChunk queries of one query group: grid
+// (chunks, BH), 8 warps, one query per warp at a time; the chunk's votes are
+// added to the group's (integer atomics: the totals do not depend on order),
+// so a large group is spread over many CTAs.
 template <int KPL>
 __global__ void __launch_bounds__(kPqVoteThreads) pq_votes_kernel(PqArgs a) {
-  extern __shared__ uint8_t pq_sm[];
+  extern __shared__ __align__(16) uint8_t pq_sm[];
   const int M = a.d / kPqSub, Ck = a.Ck;
   float* T = reinterpret_cast<float*>(pq_sm);      // [M][16][16] codeword inner products
   float* cbq = T + M * kPqKc * kPqKc;              // [M][16][8] query codebook
-  int* wsz = reinterpret_cast<int*>(cbq + M * kPqKc * kPqSub);  // [Ck] key-group sizes
-  int* votes_s = wsz + Ck;                         // [Ck]
-  int* hist = votes_s + Ck;                        // [8 warps][256]
-  uint8_t* kc_s = reinterpret_cast<uint8_t*>(hist + 8 * 256);  // [Ck][M] key-group codes
-  const int i = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the two int arrays are padded to a multiple of 4 entries so that the
+  // code rows after them start on a 16-byte boundary (16- or 8-byte loads)
+  const int Ck4 = (Ck + 3) & ~3;
+  int* wsz = reinterpret_cast<int*>(cbq + M * kPqKc * kPqSub);  // [Ck4] key-group sizes
+  int* votes_s = wsz + Ck4;                        // [Ck4]
+  uint8_t* kc_s = reinterpret_cast<uint8_t*>(votes_s + Ck4);  // [Ck][M] key-group codes
+  const int bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __shared__ int s_work[2];  // query group, chunk within it
+  const int32_t* qoff = a.q_offsets + (size_t)bh * (a.Cq + 1);
+  if (warp == 0) {
+    const int t_glob = blockIdx.x;
+    int run = 0, found_g = -1, found_c = 0;
+    for (int c0 = 0; c0 < a.Cq && found_g < 0; c0 += 32) {
+      const int c = c0 + lane;
+      const int nc = (c < a.Cq) ? (max(qoff[c + 1] - qoff[c], 0) + kPqChunk - 1) / kPqChunk : 0;
+      int incl = nc;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const int excl = run + incl - nc;
+      const bool mine = nc > 0 && t_glob >= excl && t_glob < excl + nc;
+      const unsigned hit = __ballot_sync(0xffffffffu, mine);
+      if (hit) {
+        const int src = __ffs(hit) - 1;
+        found_g = __shfl_sync(0xffffffffu, c, src);
+        found_c = __shfl_sync(0xffffffffu, t_glob - excl, src);
+      }
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      s_work[0] = found_g;
+      s_work[1] = found_c;
+    }
+  }
+  __syncthreads();
+  const int i = s_work[0];
+  if (i < 0) return;  // chunk index beyond this head's chunks
   const float* cbh = a.codebooks + (size_t)bh * 2 * M * kPqKc * kPqSub;
   for (int t = tid; t < M * kPqKc * kPqKc; t += kPqVoteThreads) {
     const int m = t / (kPqKc * kPqKc), qa = (t / kPqKc) % kPqKc, kb = t % kPqKc;
@@ -164,10 +194,23 @@ __global__ void __launch_bounds__(kPqVoteThreads) pq_votes_kernel(PqArgs a) {
   __syncthreads();
 
   const int kcq = a.Cq < kPqKc ? a.Cq : kPqKc;
-  const int32_t* qoff = a.q_offsets + (size_t)bh * (a.Cq + 1);
-  const int qlo = qoff[i], qhi = qoff[i + 1];
-  int* h = hist + warp * 256;
+  const int qlo = qoff[i] + s_work[1] * kPqChunk, qhi = min(qoff[i + 1], qlo + kPqChunk);
   const long long E = a.E;
+  // A query's votes depend only on its codes: each warp keeps the last code
+  // vector and the key groups it voted for (bit k of a lane's mask: group
+  // lane + 32k), and a run of queries with equal codes is added as a count.
+  bool has_prev = false;
+  unsigned long long prev_cv = 0ull;
+  unsigned long long vmask = 0ull;  // KPL <= 64 bits
+  int run = 0;
+  auto flush = [&]() {
+    if (run > 0) {
+#pragma unroll
+      for (int k = 0; k < KPL; ++k)
+        if ((vmask >> k) & 1ull) atomicAdd(&votes_s[lane + 32 * k], run);
+    }
+    run = 0;
+  };
   for (int slot = qlo + warp; slot < qhi; slot += kPqVoteThreads / 32) {
     const int tok = a.q_perm[(size_t)bh * a.N + slot];
     if (tok < 0 || tok >= a.N) {  // the same for every lane
@@ -189,85 +232,107 @@ __global__ void __launch_bounds__(kPqVoteThreads) pq_votes_kernel(PqArgs a) {
       code = pq_nearest(x, cbq + lane * kPqKc * kPqSub, kcq);
     }
     int am[16];
+    unsigned long long cv = 0ull;  // the codes, 4 bits each
 #pragma unroll
-    for (int m = 0; m < 16; ++m) am[m] = __shfl_sync(0xffffffffu, code, m);
-    // rank keys of this lane's key groups j = lane + 32k (0: empty or absent)
-    unsigned long long key[KPL];
+    for (int m = 0; m < 16; ++m) {
+      am[m] = __shfl_sync(0xffffffffu, code, m);
+      if (m < M) cv |= (unsigned long long)am[m] << (4 * m);
+    }
+    if (has_prev && cv == prev_cv) {
+      ++run;
+      continue;
+    }
+    flush();
+    // score order of this lane's key groups j = lane + 32k (weight 0: empty or absent)
+    uint32_t so[KPL];
+    int wk[KPL];
+    uint32_t top = 0u;
 #pragma unroll
     for (int k = 0; k < KPL; ++k) {
       const int j = lane + 32 * k;
-      key[k] = 0ull;
+      so[k] = 0u;
+      wk[k] = 0;
       if (j < Ck && wsz[j] > 0) {
-        float s = 0.0f;
+        // the group's M codes in one 16-byte (d = 128) or 8-byte (d = 64) load
+        uint4 cw = make_uint4(0u, 0u, 0u, 0u);
+        if (M == 16) {
+          cw = *reinterpret_cast<const uint4*>(kc_s + j * 16);
+        } else {
+          const uint2 c2 = *reinterpret_cast<const uint2*>(kc_s + j * 8);
+          cw.x = c2.x;
+          cw.y = c2.y;
+        }
+        const uint32_t cwv[4] = {cw.x, cw.y, cw.z, cw.w};
+        float sc = 0.0f;
 #pragma unroll
         for (int m = 0; m < 16; ++m)
-          if (m < M) s = __fadd_rn(s, T[(m * kPqKc + am[m]) * kPqKc + kc_s[j * M + m]]);
-        key[k] = ((unsigned long long)pq_float_order(s) << 12) | (unsigned)(4095 - j);
+          if (m < M) sc = __fadd_rn(sc, T[(m * kPqKc + am[m]) * kPqKc + ((cwv[m >> 2] >> (8 * (m & 3))) & 0xFFu)]);
+        so[k] = pq_float_order(sc);  // >= 0x007FFFFF for a finite score
+        wk[k] = wsz[j];
+        top = max(top, so[k]);
       }
     }
-    // weighted radix select of the first rank that does not fit
-    unsigned long long prefix = 0ull, mask = 0ull;
-    long long above = 0;  // weight of the keys above the current range
-    bool all_fit = false;
-#pragma unroll 1
-    for (int pass = 0; pass < 6; ++pass) {
-      const int sh = pass < 5 ? 36 - 8 * pass : 0;
-      const unsigned dmask = pass < 5 ? 0xFFu : 0xFu;
-      for (int b = lane; b < 256; b += 32) h[b] = 0;
-      __syncwarp();
+    // Budget prefix in rank order (score descending, then lower j): the
+    // groups strictly above the boundary score level (binary search for the
+    // smallest level u with W(score order >= u) <= E), then the groups at the
+    // boundary level in j order while they fit (rank 0 always).
+    auto W_ge = [&](uint32_t u) -> long long {
+      unsigned w = 0u;
+#pragma unroll
+      for (int k = 0; k < KPL; ++k) w += so[k] >= u ? (unsigned)wk[k] : 0u;  // empty: weight 0
+      return (long long)__reduce_add_sync(0xffffffffu, w);
+    };
+    vmask = 0ull;
+    if (W_ge(1u) <= E) {  // every group fits
 #pragma unroll
       for (int k = 0; k < KPL; ++k)
-        if (key[k] != 0ull && (key[k] & mask) == prefix)
-          atomicAdd(&h[(unsigned)(key[k] >> sh) & dmask], wsz[lane + 32 * k]);
-      __syncwarp();
-      int hb[8];
-      long long lane_total = 0;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        hb[t] = h[8 * lane + t];
-        lane_total += hb[t];
-      }
-      // weight of the bins held by higher lanes (better keys)
-      long long higher = lane_total;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const long long v = __shfl_down_sync(0xffffffffu, higher, o);
-        if (lane + o < 32) higher += v;
-      }
-      higher -= lane_total;
-      // this lane's highest bin where the running weight from the top passes E
-      int cand = -1;
-      long long cand_above = 0, run = above + higher;
-#pragma unroll
-      for (int t = 7; t >= 0; --t) {
-        const long long before = run;
-        run += hb[t];
-        if (cand < 0 && run > E) {
-          cand = 8 * lane + t;
-          cand_above = before;
+        if (wk[k] > 0) vmask |= 1ull << k;
+    } else {
+      uint32_t lo = 1u, hi = __reduce_max_sync(0xffffffffu, top) + 1u;  // W(>= lo) > E >= W(>= hi) = 0
+      long long w_hi = 0;
+#pragma unroll 1
+      while (hi - lo > 1u) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        const long long w = W_ge(mid);
+        if (w > E) {
+          lo = mid;
+        } else {
+          hi = mid;
+          w_hi = w;
         }
       }
-      const int delta = __reduce_max_sync(0xffffffffu, cand);
-      if (delta < 0) {
-        all_fit = true;
-        break;
-      }
-      above = __shfl_sync(0xffffffffu, cand_above, delta >> 3);
-      prefix |= (unsigned long long)delta << sh;
-      mask |= (unsigned long long)dmask << sh;
-      __syncwarp();
-    }
-    // votes: keys above kappa = prefix; the top key alone when none is above
 #pragma unroll
-    for (int k = 0; k < KPL; ++k) {
-      if (key[k] == 0ull) continue;
-      if (all_fit || key[k] > prefix || (above == 0 && key[k] == prefix)) atomicAdd(&votes_s[lane + 32 * k], 1);
+      for (int k = 0; k < KPL; ++k)
+        if (wk[k] > 0 && so[k] >= hi) vmask |= 1ull << k;
+      // boundary level lo, in ascending j
+      long long acc = w_hi;
+      bool stop = false;
+#pragma unroll
+      for (int k = 0; k < KPL; ++k) {
+        unsigned tied = __ballot_sync(0xffffffffu, wk[k] > 0 && so[k] == lo);
+        while (tied != 0u && !stop) {
+          const int src = __ffs(tied) - 1;
+          tied &= tied - 1u;
+          const long long w = __shfl_sync(0xffffffffu, wk[k], src);
+          if (acc == 0 || acc + w <= E) {  // acc == 0: nothing ranks above, rank 0 is kept
+            acc += w;
+            if (lane == src) vmask |= 1ull << k;
+          } else {
+            stop = true;
+          }
+        }
+        if (stop) break;
+      }
     }
-    __syncwarp();
+    prev_cv = cv;
+    has_prev = true;
+    run = 1;
   }
+  flush();
   __syncthreads();
   int32_t* vout = a.votes + ((size_t)bh * a.Cq + i) * Ck;
-  for (int j = tid; j < Ck; j += kPqVoteThreads) vout[j] = votes_s[j];
+  for (int j = tid; j < Ck; j += kPqVoteThreads)
+    if (votes_s[j] != 0) atomicAdd(vout + j, votes_s[j]);
 }
 
 size_t pq_scratch_bytes(int BH, int d, int Ck) {
@@ -283,17 +348,20 @@ cudaError_t launch_pq_votes(const PqArgs& a0, void* scratch, cudaStream_t s) {
   a.codebooks = reinterpret_cast<float*>(scratch);
   const size_t cb = (size_t)a.BH * 2 * M * kPqKc * kPqSub * sizeof(float);
   a.kcodes = reinterpret_cast<uint8_t*>(scratch) + (cb + 255) / 256 * 256;
+  cudaError_t z = cudaMemsetAsync(a.votes, 0, (size_t)a.BH * a.Cq * a.Ck * sizeof(int32_t), s);
+  if (z != cudaSuccess) return z;
   const int cmax = a.Cq > a.Ck ? a.Cq : a.Ck;
   pq_codebook_kernel<<<dim3(M, 2, a.BH), kPqCbThreads, (size_t)cmax, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t sm = (size_t)M * kPqKc * kPqKc * 4 + (size_t)M * kPqKc * kPqSub * 4 + (size_t)a.Ck * 8 + 8 * 256 * 4 +
-                    (size_t)a.Ck * M;
+  const size_t Ck4 = ((size_t)a.Ck + 3) & ~(size_t)3;
+  const size_t sm = (size_t)M * kPqKc * kPqKc * 4 + (size_t)M * kPqKc * kPqSub * 4 + Ck4 * 8 + (size_t)a.Ck * M;
   const int kpl = (a.Ck + 31) / 32;
   auto go = [&](auto kern) -> cudaError_t {
     cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (r != cudaSuccess) return r;
-    kern<<<dim3(a.Cq, a.BH), kPqVoteThreads, sm, s>>>(a);
+    // chunks per head <= ceil(N / chunk) + Cq (one ragged chunk per group)
+    kern<<<dim3((a.N + kPqChunk - 1) / kPqChunk + a.Cq, a.BH), kPqVoteThreads, sm, s>>>(a);
     return cudaGetLastError();
   };
   if (kpl <= 4) return go(pq_votes_kernel<4>);
