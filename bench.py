@@ -282,7 +282,10 @@ def main():
     acc = {s: 0.0 for s in stages}
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
     barrier()
-    for _ in range(args.steps):
+    # one untimed pass first: the staged calls allocate their outputs, and a
+    # first allocation that blocks the host would sit inside a stage's events
+    for it in range(args.steps + 1):
+        timed = it > 0
         evs[0].record(stream)
         cq, qa, qp, qo = ig.cluster(Q, w.Cq, w.iters, p)
         evs[1].record(stream)
@@ -300,7 +303,7 @@ def main():
         evs[len(stages)].record(stream)
         torch.cuda.synchronize()
         for i, s in enumerate(stages):
-            acc[s] += evs[i].elapsed_time(evs[i + 1])
+            acc[s] += evs[i].elapsed_time(evs[i + 1]) if timed else 0.0
         del cq, qa, qp, qo, ck, ka, kp, ko, Kp, Vp, eg, cnt, sp, sb
     ig.device_status()
     stage_ms = {s: acc[s] / args.steps for s in stages}

@@ -140,3 +140,33 @@ def test_forward_pq_vote_equals_its_stages(case):
     ic = ig.forward_intermediates(wc, pc)
     assert torch.equal(ic["cq"], it["cq"]) and torch.equal(ic["k_offsets"], it["k_offsets"])
     ig.device_status()
+
+
+def test_full_size_heads_votes_bit_exact(oracle_mod):
+    """Wan2.1-14B 720p shape (N=75600, d=128, Cq=100, Ck=500, 16%+16%), heads 0
+    and 39: votes and vote-ranked selections from the oracle's (one-iteration)
+    centroids and permutations, bit-exact."""
+    w = workloads.WAN14B_720P
+    heads = [0, w.H - 1]
+    Q, K, V = workloads.make_inputs(w, heads=heads)
+    p = ig.make_params(1, len(heads), w.N, w.d, w.Cq, w.Ck, iters=1, exact_frac=w.exact_frac,
+                       sample_frac=w.sample_frac, seed=77, layer=0, selection="pq_vote")
+    E = oracle_mod.budget(w.exact_frac, w.N)
+    hr, votes = [], []
+    for h in range(len(heads)):
+        f = lambda t: np_(t[0, h].float())
+        r = oracle_mod.forward_head(f(Q), f(K), f(V), Cq=w.Cq, Ck=w.Ck, iters=1, exact_frac=w.exact_frac,
+                                    sample_frac=w.sample_frac, scale=p.softmax_scale, seed=p.seed, layer=0, bh=h,
+                                    rows=[], selection="pq_vote")
+        hr.append(r)
+        votes.append(oracle_mod.pq_votes(f(Q), r.cq, r.ck, r.q_perm, r.q_offsets, r.k_offsets, E))
+    votes = np.stack(votes)
+    got = ig.pq_votes(Q.cuda(), _stack(hr, "cq"), _stack(hr, "ck"), _stack(hr, "q_perm"), _stack(hr, "q_offsets"),
+                      _stack(hr, "k_offsets"), p)
+    assert np.array_equal(np_(got)[0], votes)
+    eg, cnt, sp, sb = ig.select_sample(_stack(hr, "cq"), _stack(hr, "ck"), _stack(hr, "k_offsets"), p, votes=got)
+    for h in range(len(heads)):
+        assert np.array_equal(np_(cnt)[0, h], hr[h].counts)
+        assert np.array_equal(np_(eg)[0, h], hr[h].exact_groups)
+        assert np.array_equal(np_(sp)[0, h], hr[h].sample_pos)
+    ig.device_status()
