@@ -204,6 +204,29 @@ def reference_arm(args, w, exact, sample):
     return 0
 
 
+def max_over_ranks(vals, dist=None, device="cpu"):
+    """Element-wise maximum over all ranks of a list of per-rank floats (the
+    list itself with one rank); every rank gets the same result."""
+    if dist is None:
+        return [float(v) for v in vals]
+    import torch
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_time(t_total_ms, e2e_ms_per_call, steps, world, dist=None, device="cpu"):
+    """Whole-job timing of `world` replicas that each ran `steps` calls: the
+    slowest rank's device time sets the job's time, so
+    ms_call = max(t_total) / steps is one rank's time per call and the
+    aggregate ms per call is ms_call / world (world calls per step); the end
+    to end time per call is aggregated the same way.  Returns
+    (ms_call, aggregate ms/call, aggregate e2e ms/call)."""
+    t_max, e2e_max = max_over_ranks([t_total_ms, e2e_ms_per_call], dist, device)
+    ms_call = t_max / steps
+    return ms_call, ms_call / world, e2e_max / world
+
+
 def workload_config(w, exact, sample, selection="centroid"):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "Cq": w.Cq, "Ck": w.Ck,
             "kmeans_iters": w.iters, "exact_frac": exact, "sample_frac": sample, "sampling": "importance",
@@ -395,15 +418,9 @@ def main():
         del hQ, hK, hV, hO, hws
 
     # ---------------- max over ranks
-    t_max = t_fwd
-    if dist is not None:
-        tt = torch.tensor([t_fwd, e2e["value"] if e2e else 0.0], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt[0])
-        if e2e:
-            e2e["value"] = float(tt[1])
-    ms_call = t_max / args.steps
-    value = ms_call / world
+    ms_call, value, e2e_value = job_time(t_fwd, e2e["value"] if e2e else 0.0, args.steps, world, dist, dev)
+    if e2e:
+        e2e["value"] = e2e_value
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not pq:  # the sample runs the centroid ranking
