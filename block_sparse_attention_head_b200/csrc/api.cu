@@ -242,10 +242,14 @@ int forward_impl(const void* Q, const void* K, const void* V, void* O, const ins
 
 
 // ------------------------------------------------------ host-buffer pipeline
+// Staging slots of the host-buffer pipeline: chunk c uses slot c % 3, so the
+// copy in of chunk c + 1 never waits for the compute of chunk c - 1.
+constexpr int kHostSlots = 3;
+
 struct HostLayout {
   int hc;                 // heads per chunk (at most)
   size_t tensor;          // bytes of one chunk of one tensor (256-aligned)
-  size_t fwd_off, fwd;    // instagen_forward workspace of one chunk (two of them)
+  size_t fwd_off, fwd;    // instagen_forward workspace of one chunk (one per slot)
   size_t total;
 };
 
@@ -265,9 +269,9 @@ int host_layout(const instagen_params* p, int heads_per_chunk, HostLayout* L) {
   if (rc) return rc;
   L->hc = hc;
   L->tensor = align256((size_t)hc * head_bytes);
-  L->fwd_off = 8 * L->tensor;  // two slots x (Q, K, V, O)
+  L->fwd_off = 4 * kHostSlots * L->tensor;  // slots x (Q, K, V, O)
   L->fwd = fl.total;
-  L->total = L->fwd_off + 2 * align256(fl.total);
+  L->total = L->fwd_off + kHostSlots * align256(fl.total);
   return IG_OK;
 }
 
@@ -464,13 +468,14 @@ int instagen_forward_host(const void* Q, const void* K, const void* V, void* O, 
   if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return IG_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaStream_t s_in = nullptr, s_out = nullptr, s_c1 = nullptr;
-  cudaEvent_t ev[10] = {};  // start, in[2], comp[2], out[2], in done, out done, compute-1 done
+  constexpr int kEv = 4 + 3 * kHostSlots;  // start, in[], comp[], out[], in done, out done, compute-1 done
+  cudaEvent_t ev[kEv] = {};
   bool ok = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) == cudaSuccess &&
             cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) == cudaSuccess &&
             cudaStreamCreateWithFlags(&s_c1, cudaStreamNonBlocking) == cudaSuccess;
-  for (int i = 0; i < 10 && ok; ++i) ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
-  cudaEvent_t ev_start = ev[0], *ev_in = ev + 1, *ev_comp = ev + 3, *ev_out = ev + 5;
-  cudaEvent_t ev_in_done = ev[7], ev_out_done = ev[8], ev_c1_done = ev[9];
+  for (int i = 0; i < kEv && ok; ++i) ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+  cudaEvent_t ev_start = ev[0], *ev_in = ev + 1, *ev_comp = ev + 1 + kHostSlots, *ev_out = ev + 1 + 2 * kHostSlots;
+  cudaEvent_t ev_in_done = ev[kEv - 3], ev_out_done = ev[kEv - 2], ev_c1_done = ev[kEv - 1];
   // chunks alternate between two compute streams (the caller's and one of
   // ours), each with its own forward workspace, so one chunk's tail overlaps
   // the next chunk's first kernels
@@ -487,37 +492,41 @@ int instagen_forward_host(const void* Q, const void* K, const void* V, void* O, 
          cudaStreamWaitEvent(s_c1, ev_start, 0) == cudaSuccess;
     if (!ok) rc = IG_ERR_CUDA;
   }
-  // chunk sizes of a batch row: a small first chunk (short pipeline fill),
-  // then hc heads, and a small last chunk (short drain)
-  const int q = L.hc / 4 > 1 ? L.hc / 4 : 1;
-  auto chunk_at = [&](int h) {
+  // chunk sizes of a batch row: one head first, so the GPU starts after one
+  // head's copy in; then each chunk half again as large as the one before, up
+  // to hc, so that (the copy in of a head being faster than its compute) the
+  // next chunk is in before this one is computed; and one head last, a short
+  // drain.  Small chunks cost a little (smaller grids, more launches), the
+  // growth keeps their number logarithmic in hc.
+  auto chunk_at = [&](int h, int prev) {
     const int left = p->H - h;
-    if (h == 0) return left < q ? left : q;
-    if (left <= q) return left;
-    if (left <= L.hc + q) return left - q;
-    return L.hc;
+    if (h == 0 || left <= 1) return 1;
+    int n = (3 * prev + 1) / 2;
+    if (n < prev + 1) n = prev + 1;
+    if (n > L.hc) n = L.hc;
+    return left <= n + 1 ? left - 1 : n;
   };
   int c = 0;
   for (int b = 0; b < p->B && rc == IG_OK; ++b) {
     for (int h0 = 0, n = 0; h0 < p->H && rc == IG_OK; h0 += n, ++c) {
-      n = chunk_at(h0);
-      const int slot = c & 1;
+      n = chunk_at(h0, n);
+      const int slot = c % kHostSlots;
       const size_t off = ((size_t)b * p->H + h0) * head_bytes, bytes = (size_t)n * head_bytes;
       char* dq = w + (4 * slot + 0) * L.tensor;
       char* dk = w + (4 * slot + 1) * L.tensor;
       char* dv = w + (4 * slot + 2) * L.tensor;
       char* dout = w + (4 * slot + 3) * L.tensor;
-      // copy in: the slot's inputs are free once chunk c - 2 is computed
-      ok = (c < 2 || cudaStreamWaitEvent(s_in, ev_comp[slot], 0) == cudaSuccess) &&
+      // copy in: the slot's inputs are free once chunk c - kHostSlots is computed
+      ok = (c < kHostSlots || cudaStreamWaitEvent(s_in, ev_comp[slot], 0) == cudaSuccess) &&
            cudaMemcpyAsync(dq, hq + off, bytes, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
            cudaMemcpyAsync(dk, hk + off, bytes, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
            cudaMemcpyAsync(dv, hv + off, bytes, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
            cudaEventRecord(ev_in[slot], s_in) == cudaSuccess;
-      // compute (stream of this slot): after the copy in, and once chunk
-      // c - 2's output left the slot
-      cudaStream_t cs = slot ? s_c1 : s;
+      // compute (consecutive chunks alternate between two streams): after
+      // the copy in, and once chunk c - kHostSlots's output left the slot
+      cudaStream_t cs = (c & 1) ? s_c1 : s;
       ok = ok && cudaStreamWaitEvent(cs, ev_in[slot], 0) == cudaSuccess &&
-           (c < 2 || cudaStreamWaitEvent(cs, ev_out[slot], 0) == cudaSuccess);
+           (c < kHostSlots || cudaStreamWaitEvent(cs, ev_out[slot], 0) == cudaSuccess);
       if (!ok) {
         rc = IG_ERR_CUDA;
         break;
@@ -542,7 +551,7 @@ int instagen_forward_host(const void* Q, const void* K, const void* V, void* O, 
   if (s_out && ev_out_done && cudaEventRecord(ev_out_done, s_out) == cudaSuccess)
     cudaStreamWaitEvent(s, ev_out_done, 0);
   if (s_c1 && ev_c1_done && cudaEventRecord(ev_c1_done, s_c1) == cudaSuccess) cudaStreamWaitEvent(s, ev_c1_done, 0);
-  for (int i = 0; i < 10; ++i)
+  for (int i = 0; i < kEv; ++i)
     if (ev[i]) cudaEventDestroy(ev[i]);  // released once their work completes
   if (s_in) cudaStreamDestroy(s_in);
   if (s_out) cudaStreamDestroy(s_out);

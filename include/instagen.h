@@ -278,21 +278,24 @@ int instagen_forward_init(const void* Q, const void* K, const void* V, void* O, 
  * instagen_forward with HOST buffers: Q, K, V (inputs) and O (output) are
  * host memory in the [B,H,N,d] bf16 layout of instagen_forward.  No
  * counterpart on the method's pages: the heads are independent, so the call
- * splits them into chunks of heads_per_chunk consecutive heads of one batch
- * row (0: chosen by the library, about 160 MB per tensor per chunk; the
- * first and last chunks of a row are a quarter of that) and pipelines them:
- * while chunk c is computed, chunk c + 1 is copied in on one copy stream and
- * chunk c - 1 copied out on another, so the PCIe transfers overlap the
- * kernels.  The result equals instagen_forward on
+ * splits them into chunks of at most heads_per_chunk consecutive heads of
+ * one batch row (0: chosen by the library, about 160 MB per tensor per
+ * chunk) and pipelines them: while chunk c is computed, the next chunks are
+ * copied in on one copy stream and chunk c - 1 copied out on another, so the
+ * PCIe transfers overlap the kernels.  A row's first chunk is one head (the
+ * kernels start after one head's copy), each next chunk half again as large
+ * as the one before up to heads_per_chunk (its copy in then ends before the
+ * chunk in front of it is computed), and its last chunk one head (a short
+ * drain).  The result equals instagen_forward on
  * device copies of the same inputs, bit for bit (every head draws its sample
  * with its global head index).
  *   Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister);
  *   pageable memory works but the copies then do not overlap.
  *   ws >= instagen_forward_host_workspace_size(p, heads_per_chunk) bytes of
- *   DEVICE memory, 256-B aligned: two staging slots for a chunk's Q, K, V and
- *   O plus two of instagen_forward's workspaces for one chunk (consecutive
- *   chunks run on two compute streams, `stream` and an internal one, so one
- *   chunk's last kernels overlap the next chunk's first).
+ *   DEVICE memory, 256-B aligned: three staging slots, each a chunk's Q, K,
+ *   V and O plus one of instagen_forward's workspaces for one chunk
+ *   (consecutive chunks run on two compute streams, `stream` and an internal
+ *   one, so one chunk's last kernels overlap the next chunk's first).
  *   Everything is enqueued asynchronously; `stream` is ordered after all of
  *   it (synchronise it before reading O).  The internal streams and their
  *   events are created and released inside the call, so it must not run

@@ -98,8 +98,8 @@ def test_null_pointers_and_workspace_rejected(lib):
 def test_forward_host_checks_on_host(lib):
     p = ig.make_params(2, 5, 1000, 128, 8, 16)
     L1 = lib.instagen_workspace_size(ctypes.byref(ig.make_params(1, 2, 1000, 128, 8, 16)))
-    # two staging slots of 2 heads x (Q, K, V, O) plus one chunk's forward workspace
-    assert lib.instagen_forward_host_workspace_size(ctypes.byref(p), 2) >= 8 * 2 * 1000 * 128 * 2 + L1
+    # three staging slots, each 2 heads x (Q, K, V, O) and one chunk's forward workspace
+    assert lib.instagen_forward_host_workspace_size(ctypes.byref(p), 2) >= 3 * (4 * 2 * 1000 * 128 * 2 + L1)
     assert lib.instagen_forward_host_workspace_size(ctypes.byref(p), -1) == 0
     # automatic chunk: all 5 small heads in one chunk
     L5 = lib.instagen_workspace_size(ctypes.byref(ig.make_params(1, 5, 1000, 128, 8, 16)))

@@ -354,16 +354,17 @@ def test_forward_warm_start():
 def test_forward_host_pipeline_equals_forward():
     """instagen_forward_host (host buffers, head chunks pipelined over three
     streams) gives exactly the device-buffer call's output: every head draws
-    its sample with its global head index.  B = 2, H = 3 in chunks of 2 heads
-    -> 4 chunks (two per batch row, one ragged), so both staging slots are
-    reused."""
-    B, H, N, d = 2, 3, 1000, 128
+    its sample with its global head index.  B = 2, H = 5 in chunks of at most
+    2 heads -> rows of chunks 1, 2, 1, 1 (8 chunks), so every one of the three
+    staging slots is reused; the library's own chunking and one-head chunks
+    too."""
+    B, H, N, d = 2, 5, 1000, 128
     Q, K, V = workloads.random_small(41, N, d, n_centres=12, sigma=0.4, H=B * H)
     Q, K, V = (t.reshape(B, H, N, d).contiguous() for t in (Q, K, V))
     p = ig.make_params(B, H, N, d, 7, 40, iters=3, exact_frac=0.2, sample_frac=0.1, seed=77, layer=2)
     ref = ig.forward(Q.cuda(), K.cuda(), V.cuda(), p)
     hQ, hK, hV = (t.pin_memory() for t in (Q, K, V))
-    for hpc in (2, 0):
+    for hpc in (2, 0, 1):
         O = ig.forward_host(hQ, hK, hV, p, heads_per_chunk=hpc)
         torch.cuda.current_stream().synchronize()
         assert torch.equal(O, ref.cpu()), f"heads_per_chunk={hpc}"
