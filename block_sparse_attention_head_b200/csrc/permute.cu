@@ -20,11 +20,17 @@ namespace ig {
 // starts and the number of earlier tokens of each cluster in lower-ranked
 // CTAs; phase 3 walks each warp range in order (32 tokens at a time, ranks
 // inside a step from __match_any_sync), so equal clusters keep ascending
-// token index.  The sort is a single launch and needs no global scratch.
+// token index.  The first kSortRegs steps of a warp's range stay in registers
+// from phase 1 to phase 3 (all their loads in flight at once; the ordered walk
+// then waits on no memory); longer ranges read the rest again.  The sort is a
+// single launch and needs no global scratch.
 constexpr int kSortMaxCtas = 8;
 constexpr int kSortUnroll = 4;
+constexpr int kSortRegs = 40;     // 32-token steps per warp held in registers
+constexpr int kSortMaxWarps = 8;   // 256 threads, 3 CTAs per SM: 55 heads of 8 CTAs in one wave
 
-__global__ void count_sort_kernel(const int32_t* __restrict__ assign, int N, int C, int32_t* __restrict__ perm,
+__global__ void __launch_bounds__(kSortMaxWarps * 32, 3)
+    count_sort_kernel(const int32_t* __restrict__ assign, int N, int C, int32_t* __restrict__ perm,
                                   int32_t* __restrict__ offsets) {
   extern __shared__ int sort_smem[];  // cnt [nwarps][C], ctot [C], before [C], base [C+1]
   namespace cg = cooperative_groups;
@@ -44,7 +50,23 @@ __global__ void count_sort_kernel(const int32_t* __restrict__ assign, int N, int
   const int q0 = (int)((long long)N * r / S), q1 = (int)((long long)N * (r + 1) / S);
   const int seg = (q1 - q0 + nwarps - 1) / nwarps;
   const int s0 = min(q1, q0 + warp * seg), s1 = min(q1, s0 + seg);
-  for (int i0 = s0 + lane; i0 < s1; i0 += 32 * kSortUnroll) {
+  const int sreg = min(s1, s0 + 32 * kSortRegs);  // end of the register-held part
+  int vr[kSortRegs];
+#pragma unroll
+  for (int k = 0; k < kSortRegs; ++k) {
+    const int i = s0 + 32 * k + lane;
+    vr[k] = i < sreg ? a[i] : -1;
+  }
+#pragma unroll
+  for (int k = 0; k < kSortRegs; ++k) {
+    if (s0 + 32 * k + lane < sreg) {
+      if (vr[k] >= 0 && vr[k] < C)
+        atomicAdd(&cnt[warp * C + vr[k]], 1);
+      else
+        raise_error(kErrIndex);
+    }
+  }
+  for (int i0 = sreg + lane; i0 < s1; i0 += 32 * kSortUnroll) {
     int v[kSortUnroll];
 #pragma unroll
     for (int u = 0; u < kSortUnroll; ++u) v[u] = (i0 + 32 * u < s1) ? a[i0 + 32 * u] : 0;
@@ -104,11 +126,9 @@ __global__ void count_sort_kernel(const int32_t* __restrict__ assign, int N, int
   }
   __syncthreads();
   const unsigned lt_mask = (1u << lane) - 1u;
-  int nxt = (s0 + lane < s1) ? a[s0 + lane] : -1;
-  for (int i0 = s0; i0 < s1; i0 += 32) {
-    const int i = i0 + lane;
-    int c = nxt;
-    nxt = (i + 32 < s1) ? a[i + 32] : -1;  // next step's load in flight
+  int32_t* pout = perm + (size_t)bh * N;
+  // one 32-token step in token order: lanes of equal cluster ranked by lane
+  auto place = [&](int c, int i) {
     if (c >= C || c < 0) c = -1;
     const unsigned same = __match_any_sync(0xffffffffu, c);
     const int rank = __popc(same & lt_mask);
@@ -117,18 +137,31 @@ __global__ void count_sort_kernel(const int32_t* __restrict__ assign, int N, int
     __syncwarp();
     if (c >= 0 && rank == 0) cnt[warp * C + c] += __popc(same);
     __syncwarp();
-    if (c >= 0) perm[(size_t)bh * N + pos] = i;
+    if (c >= 0) pout[pos] = i;
+  };
+#pragma unroll
+  for (int k = 0; k < kSortRegs; ++k) {
+    const int i0 = s0 + 32 * k;
+    if (i0 >= sreg) break;  // warp-uniform
+    place(i0 + lane < sreg ? vr[k] : -1, i0 + lane);
+  }
+  int nxt = (sreg + lane < s1) ? a[sreg + lane] : -1;
+  for (int i0 = sreg; i0 < s1; i0 += 32) {
+    const int i = i0 + lane;
+    const int c = nxt;
+    nxt = (i + 32 < s1) ? a[i + 32] : -1;  // next step's load in flight
+    place(c, i);
   }
 }
 
 cudaError_t launch_count_sort(const int32_t* assign, int BH, int N, int C, int32_t* perm, int32_t* offsets,
                               cudaStream_t s) {
   // one CTA per 4096 tokens of a head, up to a cluster of 8; as many warps
-  // (<= 32) as fit 160 KB of per-warp counters
+  // (<= kSortMaxWarps) as fit 160 KB of per-warp counters
   int S = (N + 4095) / 4096;
   S = S < 1 ? 1 : (S > kSortMaxCtas ? kSortMaxCtas : S);
   int nwarps = (int)((160 * 1024) / ((size_t)C * 4));
-  nwarps = nwarps < 1 ? 1 : (nwarps > 32 ? 32 : nwarps);
+  nwarps = nwarps < 1 ? 1 : (nwarps > kSortMaxWarps ? kSortMaxWarps : nwarps);
   const size_t sm = ((size_t)nwarps * C + 3 * (size_t)C + 1) * sizeof(int);
   cudaError_t e = cudaFuncSetAttribute(count_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
