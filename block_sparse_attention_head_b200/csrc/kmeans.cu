@@ -525,9 +525,13 @@ cudaError_t launch_kmeans_assign(const KmeansGeom& g, const CUtensorMap* tmap_x,
 // cluster writes its mean at once (an empty one keeps its centroid); the
 // pieces of a larger cluster store their sums, and the CTA that arrives last
 // adds them in piece order and writes the mean.  Every sum runs in a fixed
-// order, so the centroids do not depend on scheduling.
+// order, so the centroids do not depend on scheduling.  A thread's 16-byte
+// chunks of its slot's rows are fetched with cp.async into a private ring
+// of kUpdDepth shared-memory entries, so kUpdDepth rows per slot are in
+// flight without holding registers; a thread reads only entries it copied,
+// so the ring needs no barrier, only cp.async.wait_group.
 constexpr int kUpdThreads = 256;
-constexpr int kUpdUnroll = 4;  // rows in flight per slot
+constexpr int kUpdDepth = 8;  // rows in flight per slot
 
 __device__ __forceinline__ int update_pieces(int n) { return n <= kUpdRows ? 1 : (n + kUpdRows - 1) / kUpdRows; }
 
@@ -536,7 +540,7 @@ __global__ void __launch_bounds__(kUpdThreads)
                          const int32_t* __restrict__ offsets, float* __restrict__ cent,
                          __nv_bfloat16* __restrict__ cmma, float* __restrict__ norms, float* __restrict__ partial,
                          int32_t* __restrict__ arrive, int part_slots) {
-  __shared__ float part[kUpdThreads * 8];
+  __shared__ __align__(16) uint4 ring[kUpdDepth][kUpdThreads];  // later the slot partial sums
   __shared__ int rows_s[kUpdRows];  // the piece's token indices
   __shared__ float red[32];
   __shared__ int scan_np[kUpdThreads / 32], scan_mp[kUpdThreads / 32];
@@ -607,36 +611,39 @@ __global__ void __launch_bounds__(kUpdThreads)
   for (int p = plo + tid; p < phi; p += kUpdThreads) rows_s[p - plo] = prow[p];
   __syncthreads();
   const __nv_bfloat16* xh = X + (size_t)bh * g.N * g.d + ch * 8;
+  // this slot's rows: plo + slot + slots * k, k < nk, added in that order
+  const int nk = phi - plo > slot ? (phi - plo - slot + slots - 1) / slots : 0;
+  auto issue = [&](int k) {
+    const int src = rows_s[slot + slots * k];
+    const bool ok = src >= 0 && src < g.N;
+    if (!ok) raise_error(kErrIndex);
+    cp_async_16(smem_u32(&ring[k % kUpdDepth][tid]), xh + (size_t)(ok ? src : 0) * g.d, ok ? 16u : 0u);
+  };
+#pragma unroll
+  for (int k = 0; k < kUpdDepth; ++k) {
+    if (k < nk) issue(k);
+    cp_async_commit();  // one group per row, empty past the end
+  }
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  for (int p0 = plo + slot; p0 < phi; p0 += kUpdUnroll * slots) {
-    int src[kUpdUnroll];
-    uint4 raw[kUpdUnroll];
+  for (int k = 0; k < nk; ++k) {
+    cp_async_wait<kUpdDepth - 1>();  // row k's group is the oldest of the last kUpdDepth
+    const uint4 raw = ring[k % kUpdDepth][tid];
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-    for (int u = 0; u < kUpdUnroll; ++u) {
-      const int p = p0 + u * slots;
-      src[u] = p < phi ? rows_s[p - plo] : -1;
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h2[e]);
+      acc[2 * e] += f.x;
+      acc[2 * e + 1] += f.y;
     }
-#pragma unroll
-    for (int u = 0; u < kUpdUnroll; ++u) {
-      const bool live = p0 + u * slots < phi;
-      const bool ok = src[u] >= 0 && src[u] < g.N;
-      if (live && !ok) raise_error(kErrIndex);
-      raw[u] = (live && ok) ? *reinterpret_cast<const uint4*>(xh + (size_t)src[u] * g.d) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < kUpdUnroll; ++u) {  // rows added in permuted order
-      if (p0 + u * slots >= phi) break;
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(h2[e]);
-        acc[2 * e] += f.x;
-        acc[2 * e + 1] += f.y;
-      }
-    }
+    // the entry is refilled only after its value was consumed above
+    if (k + kUpdDepth < nk) issue(k + kUpdDepth);
+    cp_async_commit();
   }
+  cp_async_wait_all();
+  __syncthreads();  // every ring read done: the ring becomes the slot sums
+  float* part = reinterpret_cast<float*>(&ring[0][0]);
 #pragma unroll
   for (int e = 0; e < 8; ++e) part[slot * g.d + ch * 8 + e] = acc[e];
   __syncthreads();
