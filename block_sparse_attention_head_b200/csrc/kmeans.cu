@@ -131,12 +131,16 @@ cudaError_t launch_kmeans_init(const KmeansGeom& g, const __nv_bfloat16* X, cons
 // heads.  Token tiles are double-buffered (the next unit streams in from HBM
 // during the current one) and the centroid halves stream through a ring of
 // K-blocks of 64 columns (TMA, 128-byte swizzle).  TMEM: 2 buffers x 256 fp32
-// columns; epilogue group b (4 warps) reduces the chunks that land in buffer
-// b, and the two groups' partial minima of a unit are merged through shared
-// memory.  Warps: 0 centroid producer, 1 TMEM owner + MMA issuer (leader
-// CTA), 2 token producer, 4-7 / 8-11 epilogue groups 0 / 1.
+// columns; epilogue group b reduces the chunks that land in buffer b, split
+// between two halves of 4 warps that take the lower and upper half of the
+// chunk's columns (16-column TMEM loads, the next in flight while one is
+// reduced): the reduction waits on TMEM loads, so twice the warps keep twice
+// the loads in flight.  A unit's partial minima merge through shared memory,
+// the upper half into the lower, then group 1 into group 0.  Warps: 0
+// centroid producer, 1 TMEM owner + MMA issuer (leader CTA), 2 token
+// producer, 4 + 8h + 4b + q: group b, half h, TMEM lane quarter q.
 namespace {
-constexpr int kAssignThreads = 384;
+constexpr int kAssignThreads = 640;
 constexpr int kAssignStages = 6;
 constexpr int kAssignXBufs = 3;  // token tiles in flight
 
@@ -148,42 +152,39 @@ struct AssignSmem {
   static constexpr int kX = 0;                              // token tile ring
   static constexpr int kStages = kX + kAssignXBufs * kXTileBytes;
   static constexpr int kMerge = kStages + kAssignStages * kStageBytes;  // [2 slots][128] (distance, index)
-  static constexpr int kNorms = kMerge + 2 * 128 * 8;                   // [8 epilogue warps][256] fp32
-  static constexpr int kBars = kNorms + 8 * 256 * 4;
-  // c_full, c_empty [stages]; x_full, x_empty [x bufs]; t_full, t_empty, m_full, m_empty [2]; fin
-  static constexpr int kNumBars = 2 * kAssignStages + 2 * kAssignXBufs + 8 + 1;
+  static constexpr int kHMerge = kMerge + 2 * 128 * 8;                  // [group][2 slots][128] (distance, index)
+  static constexpr int kNorms = kHMerge + 4 * 128 * 8;                  // [16 epilogue warps][128] fp32
+  static constexpr int kBars = kNorms + 16 * 128 * 4;
+  // c_full, c_empty [stages]; x_full, x_empty [x bufs]; t_full, t_empty, m_full, m_empty [2]; fin;
+  // h_full, h_empty [group][2]
+  static constexpr int kNumBars = 2 * kAssignStages + 2 * kAssignXBufs + 8 + 1 + 8;
   static constexpr int kMisc = kBars + kNumBars * 8;  // tmem base, abort flag
   static constexpr size_t bytes() { return 1024 + kMisc + 16; }
 };
 }  // namespace
 
-// Folds 32 distance columns into the running (best, best_j): dist =
+// Folds 16 distance columns into the running (best, best_j): dist =
 // ||c||^2 - 2 x.c with the norms `nw` (shared memory, same address in every
-// lane); columns at or past `chunk` are ignored.  Argmin by a pairwise tree in
-// which the right operand wins only when strictly smaller, so ties keep the
-// lowest index; padding centroids have an infinite norm and never win.
-__device__ __forceinline__ void assign_reduce32(float (&x)[32], const float4* nw, int cb, int chunk, int j0,
-                                                float& best, int& best_j) {
-  float4 nv[8];
+// lane).  Argmin by a pairwise tree in which the right operand wins only when
+// strictly smaller, and the running minimum is replaced only by a strictly
+// smaller one, so ties keep the lowest index; padding centroids have an
+// infinite norm and never win.
+__device__ __forceinline__ void assign_reduce16(const float (&x)[16], const float4* nw, int j0, float& best,
+                                                int& best_j) {
+  float m[8];
+  int ix[8];
 #pragma unroll
-  for (int u = 0; u < 8; ++u) nv[u] = nw[u];
-  const float* nf = reinterpret_cast<const float*>(nv);
-  if (cb + 32 > chunk) {  // columns past the chunk hold no product
-#pragma unroll
-    for (int e = 0; e < 32; ++e)
-      if (cb + e >= chunk) x[e] = 0.f;
-  }
-  float m[16];
-  int ix[16];
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const float a = fmaf(-2.f, x[2 * k], nf[2 * k]);
-    const float b = fmaf(-2.f, x[2 * k + 1], nf[2 * k + 1]);
-    ix[k] = b < a ? 2 * k + 1 : 2 * k;
-    m[k] = fminf(a, b);
+  for (int u = 0; u < 4; ++u) {
+    const float4 n = nw[u];
+    const float a0 = fmaf(-2.f, x[4 * u], n.x), a1 = fmaf(-2.f, x[4 * u + 1], n.y);
+    const float a2 = fmaf(-2.f, x[4 * u + 2], n.z), a3 = fmaf(-2.f, x[4 * u + 3], n.w);
+    ix[2 * u] = a1 < a0 ? 4 * u + 1 : 4 * u;
+    m[2 * u] = fminf(a0, a1);
+    ix[2 * u + 1] = a3 < a2 ? 4 * u + 3 : 4 * u + 2;
+    m[2 * u + 1] = fminf(a2, a3);
   }
 #pragma unroll
-  for (int w = 8; w >= 1; w >>= 1) {
+  for (int w = 4; w >= 1; w >>= 1) {
 #pragma unroll
     for (int k = 0; k < w; ++k) {
       const bool lt = m[2 * k + 1] < m[2 * k];
@@ -214,7 +215,10 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   uint64_t* m_full = t_full + 4;                // [2] per merge slot
   uint64_t* m_empty = t_full + 6;               // [2]
   uint64_t* fin = t_full + 8;
+  uint64_t* h_full = t_full + 9;    // [group * 2 + slot]
+  uint64_t* h_empty = t_full + 13;  // [group * 2 + slot]
   float2* merge = reinterpret_cast<float2*>(smem + L::kMerge);
+  float2* hmerge = reinterpret_cast<float2*>(smem + L::kHMerge);
   float4* norms_s = reinterpret_cast<float4*>(smem + L::kNorms);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
@@ -246,9 +250,13 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&t_full[b], 1);
-      mbar_init(&t_empty[b], 8);  // one epilogue group: 4 warps x 2 CTAs
+      mbar_init(&t_empty[b], 16);  // one epilogue group: 8 warps x 2 CTAs
       mbar_init(&m_full[b], 4);
       mbar_init(&m_empty[b], 4);
+    }
+    for (int b = 0; b < 4; ++b) {
+      mbar_init(&h_full[b], 4);
+      mbar_init(&h_empty[b], 4);
     }
     mbar_init(fin, 1);
     *abort_flag = 0;
@@ -385,11 +393,18 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     mbar_wait_drain(fin, 0);
   } else if (warp >= 4) {
     // ------------------------------------------------- epilogue (both)
-    const int grp = (warp - 4) >> 2;  // TMEM buffer this group reduces
+    const int ew = warp - 4;
+    const int grp = (ew >> 2) & 1;         // TMEM buffer this warp reduces
+    const int hf = ew >> 3;                // column half of the chunk
     const int r = (warp & 3) * 32 + lane;  // row of this CTA's tile = TMEM lane
     const uint32_t lane_off = (uint32_t)((r & ~31) << 16);
     const uint32_t t_empty_lead = mapa_shared(smem_u32(&t_empty[grp]), 0);
-    int gc = 0;
+    // this half's columns of a chunk, [h0, h1): multiples of 16, at most 128
+    const int hcols = (g.chunk / 2 + 15) / 16 * 16;
+    const int h0 = hf * hcols, h1 = min(g.chunk, h0 + hcols);
+    const int ncol = h1 - h0;
+    float4* nw = norms_s + ew * 32;
+    int gc = 0, hm = 0;  // global chunk counter, half merges of this group
     bool ok = true;
     for (int i = 0; i < nunits && ok; ++i) {
       const long long q = u0 + i;
@@ -400,40 +415,35 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       for (int c = 0; c < nchunks; ++c, ++gc) {
         const int b = gc & 1;
         if (b != grp) continue;
-        // ||c||^2 of the chunk, fetched before the wait and kept in this
+        // ||c||^2 of this half, fetched before the wait and kept in this
         // warp's shared-memory slice; padding centroids have an infinite norm
-        // and columns past the chunk get one, so neither can win (an
-        // infinite distance never compares below `best`)
+        // and never win (an infinite distance never compares below `best`)
         const float kInf = __int_as_float(0x7f800000);
-        const float4* nsrc = reinterpret_cast<const float4*>(nrm + c * g.chunk);
-        const float4 nl0 = (4 * lane < g.chunk) ? __ldg(nsrc + lane) : make_float4(kInf, kInf, kInf, kInf);
-        const float4 nl1 =
-            (4 * (lane + 32) < g.chunk) ? __ldg(nsrc + lane + 32) : make_float4(kInf, kInf, kInf, kInf);
+        const float4 nl = (4 * lane < ncol) ? __ldg(reinterpret_cast<const float4*>(nrm + c * g.chunk + h0) + lane)
+                                            : make_float4(kInf, kInf, kInf, kInf);
         if (!mbar_wait_warp_sleep(&t_full[b], (gc >> 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         __syncwarp();  // every lane is done with the previous chunk's norms
-        float4* nw = norms_s + (warp - 4) * 64;
-        nw[lane] = nl0;
-        nw[lane + 32] = nl1;
+        nw[lane] = nl;
         __syncwarp();
-        const uint32_t col0 = tmem + lane_off + (uint32_t)(b * 256);
-        // 32-column groups, the next group's TMEM load in flight while one is
+        const uint32_t col0 = tmem + lane_off + (uint32_t)(b * 256 + h0);
+        // 16-column groups, the next group's TMEM load in flight while one is
         // reduced (each wait covers the one load then outstanding)
-        float va[32], vb[32];
-        tmem_ld32(col0, va);
-        for (int cb = 0; cb < g.chunk; cb += 64) {
+        float va[16], vb[16];
+        if (ncol > 0) tmem_ld16(col0, va);
+        for (int cb = 0; cb < ncol; cb += 32) {
           tmem_wait_ld();
-          pin_regs32(va);
-          if (cb + 32 < g.chunk) tmem_ld32(col0 + cb + 32, vb);
-          assign_reduce32(va, nw + cb / 4, cb, g.chunk, c * g.chunk + cb, best, best_j);
-          if (cb + 32 < g.chunk) {
+          pin_regs16(va);
+          if (cb + 16 < ncol) tmem_ld16(col0 + cb + 16, vb);
+          assign_reduce16(va, nw + cb / 4, c * g.chunk + h0 + cb, best, best_j);
+          if (cb + 16 < ncol) {
             tmem_wait_ld();
-            pin_regs32(vb);
-            if (cb + 64 < g.chunk) tmem_ld32(col0 + cb + 64, va);
-            assign_reduce32(vb, nw + cb / 4 + 8, cb + 32, g.chunk, c * g.chunk + cb + 32, best, best_j);
+            pin_regs16(vb);
+            if (cb + 32 < ncol) tmem_ld16(col0 + cb + 32, va);
+            assign_reduce16(vb, nw + cb / 4 + 4, c * g.chunk + h0 + cb + 16, best, best_j);
           }
         }
         tc_fence_before();
@@ -441,18 +451,39 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         if (lane == 0) mbar_arrive_cluster(t_empty_lead);
       }
       if (!ok) break;
-      if (nchunks == 1) {
-        // one chunk per unit: the group that reduced it (units alternate
-        // between the groups) holds the whole minimum and writes it, so the
-        // two groups work on consecutive units in parallel
-        if ((gc - 1) % 2 == grp) {
-          const int tok = pr * 256 + (int)rank * 128 + r;
-          if (tok < g.N) assign[(size_t)bh * g.N + tok] = best_j;
-        }
+      // with one chunk per unit the units alternate between the groups and
+      // only the group that reduced this one holds its minimum
+      if (nchunks == 1 && (gc - 1) % 2 != grp) continue;
+      // the upper half hands its minimum to the lower half of the group; on
+      // equal distances the lower centroid index wins
+      const int hs = grp * 2 + (hm & 1);
+      float2* hslot = hmerge + hs * 128 + r;
+      if (hf == 1) {
+        if (hm >= 2 && !mbar_wait_warp_sleep(&h_empty[hs], ((hm >> 1) - 1) & 1, abort_flag)) break;
+        *hslot = make_float2(best, __int_as_float(best_j));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&h_full[hs]);
+        ++hm;
         continue;
       }
-      // merge the two groups' minima of this unit (slot i & 1); on equal
-      // distances the lower centroid index wins
+      if (!mbar_wait_warp_sleep(&h_full[hs], (hm >> 1) & 1, abort_flag)) break;
+      {
+        const float2 o = *hslot;
+        const int oj = __float_as_int(o.y);
+        if (o.x < best || (o.x == best && oj < best_j)) {
+          best = o.x;
+          best_j = oj;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&h_empty[hs]);
+      ++hm;
+      if (nchunks == 1) {
+        const int tok = pr * 256 + (int)rank * 128 + r;
+        if (tok < g.N) assign[(size_t)bh * g.N + tok] = best_j;
+        continue;
+      }
+      // merge the two groups' minima of this unit (slot i & 1)
       float2* slot = merge + (i & 1) * 128 + r;
       if (grp == 1) {
         if (i >= 2 && !mbar_wait_warp_sleep(&m_empty[i & 1], ((i >> 1) - 1) & 1, abort_flag)) break;
