@@ -561,11 +561,11 @@ cudaError_t launch_kmeans_assign(const KmeansGeom& g, const CUtensorMap* tmap_x,
 // of kUpdDepth shared-memory entries, so kUpdDepth rows per slot are in
 // flight without holding registers; a thread reads only entries it copied,
 // so the ring needs no barrier, only cp.async.wait_group.
-constexpr int kUpdThreads = 256;
 constexpr int kUpdDepth = 8;  // rows in flight per slot
 
 __device__ __forceinline__ int update_pieces(int n) { return n <= kUpdRows ? 1 : (n + kUpdRows - 1) / kUpdRows; }
 
+template <int kUpdThreads>
 __global__ void __launch_bounds__(kUpdThreads)
     kmeans_update_kernel(KmeansGeom g, const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ perm,
                          const int32_t* __restrict__ offsets, float* __restrict__ cent,
@@ -730,10 +730,17 @@ __global__ void __launch_bounds__(kUpdThreads)
 cudaError_t launch_kmeans_update(const KmeansGeom& g, const __nv_bfloat16* X, const int32_t* perm,
                                  const int32_t* offsets, float* cent, const KmeansScratch& sc, cudaStream_t s) {
   // at most C + N/R pieces per head (every cluster adds at most one piece
-  // beyond n/R); CTAs past a head's last piece return at once
+  // beyond n/R); CTAs past a head's last piece return at once.  Clusters of a
+  // few hundred rows take 128 threads: a CTA's time is then mostly the
+  // latency of its dependent loads (offsets, permutation, rows), and smaller
+  // CTAs keep more of those chains in flight per SM.
   dim3 grid(g.C + (g.N + kUpdRows - 1) / kUpdRows, g.BH);
-  kmeans_update_kernel<<<grid, kUpdThreads, 0, s>>>(g, X, perm, offsets, cent, sc.cmma, sc.norms, sc.partial,
-                                                     sc.arrive, kmeans_part_slots(g));
+  if ((long long)g.N < 512LL * g.C)
+    kmeans_update_kernel<128><<<grid, 128, 0, s>>>(g, X, perm, offsets, cent, sc.cmma, sc.norms, sc.partial,
+                                                   sc.arrive, kmeans_part_slots(g));
+  else
+    kmeans_update_kernel<256><<<grid, 256, 0, s>>>(g, X, perm, offsets, cent, sc.cmma, sc.norms, sc.partial,
+                                                   sc.arrive, kmeans_part_slots(g));
   return cudaGetLastError();
 }
 
