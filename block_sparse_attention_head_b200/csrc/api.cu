@@ -194,8 +194,12 @@ int select_impl(const float* cq, const float* ck, const int32_t* k_offsets, cons
 
 // The whole call on device buffers; bh0 = global index of the first head;
 // cq_init / ck_init: initial centroids or null (token floor(j*N/C)).
+// k_ready / v_ready (may be null): events the stream waits for before the
+// first kernel that reads K, and V, so that a caller copying Q, K and V in
+// that order can start the query clustering once Q is in.
 int forward_impl(const void* Q, const void* K, const void* V, void* O, const instagen_params* p,
-                 const float* cq_init, const float* ck_init, void* ws, size_t ws_bytes, int bh0, void* stream) {
+                 const float* cq_init, const float* ck_init, void* ws, size_t ws_bytes, int bh0, void* stream,
+                 cudaEvent_t k_ready = nullptr, cudaEvent_t v_ready = nullptr) {
   instagen_forward_layout L;
   int rc = forward_layout(p, &L);
   if (rc) return rc;
@@ -224,8 +228,10 @@ int forward_impl(const void* Q, const void* K, const void* V, void* O, const ins
   const size_t cws_bytes = L.total - L.cluster_ws;
   rc = run_cluster(Q, p->Cq, p->kmeans_iters, cq_init, p, cq, qa, qp, qo, cws, cws_bytes, s);
   if (rc) return rc;
+  if (k_ready && cudaStreamWaitEvent(s, k_ready, 0) != cudaSuccess) return IG_ERR_CUDA;
   rc = run_cluster(K, p->Ck, p->kmeans_iters, ck_init, p, ck, ka, kp, ko, cws, cws_bytes, s);
   if (rc) return rc;
+  if (v_ready && cudaStreamWaitEvent(s, v_ready, 0) != cudaSuccess) return IG_ERR_CUDA;
   rc = cuda_status(ig::launch_gather_rows(static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V),
                                           kp, p->B * p->H, p->N, p->d, Kp, Vp, false, true, s));
   if (rc) return rc;
@@ -468,13 +474,15 @@ int instagen_forward_host(const void* Q, const void* K, const void* V, void* O, 
   if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return IG_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaStream_t s_in = nullptr, s_out = nullptr, s_c1 = nullptr;
-  constexpr int kEv = 4 + 3 * kHostSlots;  // start, in[], comp[], out[], in done, out done, compute-1 done
+  // start, Q in[], K in[], V in[], comp[], out[], in done, out done, compute-1 done
+  constexpr int kEv = 4 + 5 * kHostSlots;
   cudaEvent_t ev[kEv] = {};
   bool ok = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) == cudaSuccess &&
             cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) == cudaSuccess &&
             cudaStreamCreateWithFlags(&s_c1, cudaStreamNonBlocking) == cudaSuccess;
   for (int i = 0; i < kEv && ok; ++i) ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
-  cudaEvent_t ev_start = ev[0], *ev_in = ev + 1, *ev_comp = ev + 1 + kHostSlots, *ev_out = ev + 1 + 2 * kHostSlots;
+  cudaEvent_t ev_start = ev[0], *ev_in = ev + 1, *ev_in_k = ev + 1 + kHostSlots, *ev_in_v = ev + 1 + 2 * kHostSlots;
+  cudaEvent_t *ev_comp = ev + 1 + 3 * kHostSlots, *ev_out = ev + 1 + 4 * kHostSlots;
   cudaEvent_t ev_in_done = ev[kEv - 3], ev_out_done = ev[kEv - 2], ev_c1_done = ev[kEv - 1];
   // chunks alternate between two compute streams (the caller's and one of
   // ours), each with its own forward workspace, so one chunk's tail overlaps
@@ -517,13 +525,18 @@ int instagen_forward_host(const void* Q, const void* K, const void* V, void* O, 
       char* dv = w + (4 * slot + 2) * L.tensor;
       char* dout = w + (4 * slot + 3) * L.tensor;
       // copy in: the slot's inputs are free once chunk c - kHostSlots is computed
+      // (an event after each tensor: the chunk's query clustering starts once
+      // Q is in, while K and V are still being copied)
       ok = (c < kHostSlots || cudaStreamWaitEvent(s_in, ev_comp[slot], 0) == cudaSuccess) &&
            cudaMemcpyAsync(dq, hq + off, bytes, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+           cudaEventRecord(ev_in[slot], s_in) == cudaSuccess &&
            cudaMemcpyAsync(dk, hk + off, bytes, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+           cudaEventRecord(ev_in_k[slot], s_in) == cudaSuccess &&
            cudaMemcpyAsync(dv, hv + off, bytes, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
-           cudaEventRecord(ev_in[slot], s_in) == cudaSuccess;
+           cudaEventRecord(ev_in_v[slot], s_in) == cudaSuccess;
       // compute (consecutive chunks alternate between two streams): after
-      // the copy in, and once chunk c - kHostSlots's output left the slot
+      // Q's copy in (K's and V's are waited for inside), and once chunk
+      // c - kHostSlots's output left the slot
       cudaStream_t cs = (c & 1) ? s_c1 : s;
       ok = ok && cudaStreamWaitEvent(cs, ev_in[slot], 0) == cudaSuccess &&
            (c < kHostSlots || cudaStreamWaitEvent(cs, ev_out[slot], 0) == cudaSuccess);
@@ -535,7 +548,7 @@ int instagen_forward_host(const void* Q, const void* K, const void* V, void* O, 
       pc.B = 1;
       pc.H = n;
       rc = forward_impl(dq, dk, dv, dout, &pc, nullptr, nullptr, w + L.fwd_off + slot * align256(L.fwd), L.fwd,
-                        b * p->H + h0, cs);
+                        b * p->H + h0, cs, ev_in_k[slot], ev_in_v[slot]);
       if (rc) break;
       // copy out
       ok = cudaEventRecord(ev_comp[slot], cs) == cudaSuccess &&

@@ -286,7 +286,8 @@ int instagen_forward_init(const void* Q, const void* K, const void* V, void* O, 
  * kernels start after one head's copy), each next chunk half again as large
  * as the one before up to heads_per_chunk (its copy in then ends before the
  * chunk in front of it is computed), and its last chunk one head (a short
- * drain).  The result equals instagen_forward on
+ * drain).  A chunk's Q, K and V are copied in that order and its kernels
+ * start once its Q is in.  The result equals instagen_forward on
  * device copies of the same inputs, bit for bit (every head draws its sample
  * with its global head index).
  *   Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister);
