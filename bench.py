@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-sweeps", action="store_true",
+                    help="skip the untimed budget points added to the line (density ends, sample sweep)")
     ap.add_argument("--sweep", action="store_true",
                     help="budget sweep (error vs dense SDPA and ms per call per budget, one JSON line "
                          "each) and a warm-started call; not part of the default run")
@@ -130,21 +132,26 @@ class ClockSampler:
 class OracleSample:
     """The CPU oracle on a bounded sample of the workload (one head).
 
-    Set-up (untimed): the head's inputs and one oracle k-means iteration (its
-    centroids and lists feed the timed stages).  One timed step: k-means
-    assign + update of 4096 sampled tokens against the Q and K centroids
-    (x N/4096 tokens, x iters), select/sample of the head's query groups, and
-    attention for 32 query rows (x N/32); extrapolated x B*H heads.
+    The head's inputs are drawn exactly as the GPU arm draws them (the same
+    seeded generator on the GPU when one is present, so both arms see the same
+    tensors), then copied to the host.  Set-up (untimed): one oracle k-means
+    iteration, whose centroids and lists feed the timed stages.  One timed
+    step: k-means assign + update of 4096 sampled tokens against the Q and K
+    centroids (x N/4096 tokens, x iters), select/sample of the head's query
+    groups, and attention for 32 query rows (x N/32); extrapolated x B*H heads.
     """
 
-    def __init__(self, w, exact, sample, seed=0):
+    def __init__(self, w, exact, sample, seed=0, layer=0):
         import numpy as np
         import oracle
         from block_sparse_attention_head_b200 import workloads
+        import torch
         oracle.build()
         self.np, self.oracle, self.w = np, oracle, w
-        Q, K, V = workloads.make_inputs(w, heads=[0])
-        self.Q, self.K, self.V = (t[0, 0].float().numpy() for t in (Q, K, V))
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        self.input_device = dev
+        Q, K, V = workloads.make_inputs(w, heads=[0], layer=layer, device=dev)
+        self.Q, self.K, self.V = (t[0, 0].float().cpu().numpy() for t in (Q, K, V))
         self.scale = 1.0 / math.sqrt(w.d)
         self.cq, self.qa, _ = oracle.kmeans(self.Q, w.Cq, 1)
         self.ck, self.ka, _ = oracle.kmeans(self.K, w.Ck, 1)
@@ -175,9 +182,17 @@ class OracleSample:
 
     def describe(self):
         w = self.w
-        return (f"head 0 of {w.name}: k-means assign+update of {self.n_tok} tokens for Q and K "
-                f"(x{w.N / self.n_tok:.1f} tokens, x{w.iters} iterations), select/sample of the head, "
-                f"attention on {self.n_rows} query rows (x{w.N / self.n_rows:.0f}); extrapolated x{w.B * w.H} heads")
+        return (f"head 0 of {w.name} (inputs drawn on {self.input_device} as the GPU arm draws them): k-means "
+                f"assign+update of {self.n_tok} tokens for Q and K (x{w.N / self.n_tok:.1f} tokens, x{w.iters} "
+                f"iterations), select/sample of the head, attention on {self.n_rows} query rows "
+                f"(x{w.N / self.n_rows:.0f}); extrapolated x{w.B * w.H} heads")
+
+    def fields(self):
+        """Machine-readable description of the extrapolation."""
+        w = self.w
+        return {"extrapolated": True, "heads_timed": 1, "heads_total": w.B * w.H,
+                "kmeans_tokens_timed": self.n_tok, "attention_rows_timed": self.n_rows, "tokens": w.N,
+                "input_device": self.input_device}
 
 
 def reference_arm(args, w, exact, sample):
@@ -196,7 +211,7 @@ def reference_arm(args, w, exact, sample):
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w, exact, sample),
         "cpu_baseline": {"kind": "oracle", "cores": orc.oracle.num_threads(), "sample": orc.describe(),
-                         "value": round(ms, 1), "unit": "ms/call"},
+                         "value": round(ms, 1), "unit": "ms/call", **orc.fields()},
         "e2e": {"value": round(ms, 1), "unit": "ms/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s": round(time.perf_counter() - t0, 1),
     }
@@ -225,6 +240,57 @@ def job_time(t_total_ms, e2e_ms_per_call, steps, world, dist=None, device="cpu")
     t_max, e2e_max = max_over_ranks([t_total_ms, e2e_ms_per_call], dist, device)
     ms_call = t_max / steps
     return ms_call, ms_call / world, e2e_max / world
+
+
+def budget_point(ig, Q, K, V, w, exact, sample, D, dn, *, seed, layer, reps=3, ws=None):
+    """ms per instagen_forward call (CUDA events, one warm-up, median of
+    `reps`) and the relative L2 error of its output against the dense output
+    D (||D|| = dn) for one (exact, sample) budget on the given inputs; also
+    the attended density of the call."""
+    import torch
+    p = ig.make_params(w.B, w.H, w.N, w.d, w.Cq, w.Ck, iters=w.iters, exact_frac=exact, sample_frac=sample,
+                       seed=seed, layer=layer)
+    if ws is None or ws.numel() < ig.workspace_size(p):
+        ws = torch.empty(ig.workspace_size(p), dtype=torch.uint8, device=Q.device)
+    O = torch.empty_like(Q)
+    ig.forward(Q, K, V, p, workspace=ws, out=O)
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        ig.forward(Q, K, V, p, workspace=ws, out=O)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ig.device_status()
+    err = float((O.float() - D).pow(2).sum().sqrt()) / dn
+    it = ig.forward_intermediates(ws, p)
+    cnt = it["counts"].long()
+    qoff = it["q_offsets"].long()
+    pairs = float(((qoff[..., 1:] - qoff[..., :-1]) * (cnt[..., 1] + cnt[..., 2])).sum())
+    return {"exact_frac": exact, "sample_frac": sample, "ms_per_call": round(statistics.median(ts), 3),
+            "rel_l2_vs_dense": round(err, 4), "density": round(pairs / (w.B * w.H * w.N * w.N), 4)}
+
+
+def stack_sample_sweep(ig, dev, args):
+    """The 40-layer Wan2.1-14B stack's sample-budget sweep (exact 8%, sampled
+    2 to 32%) on one full 40-head layer of it (layer 0, its own seeded
+    mixture): ms per call and error against dense attention per budget, plus
+    the exact-only call at 8%."""
+    import torch
+    import torch.nn.functional as F
+    from block_sparse_attention_head_b200 import workloads
+    ws_ = workloads.WAN14B_STACK
+    Q, K, V = workloads.make_inputs(ws_, layer=0, device=dev)
+    D = F.scaled_dot_product_attention(Q, K, V, scale=ws_.softmax_scale).float()
+    dn = float(D.pow(2).sum().sqrt())
+    pts = [budget_point(ig, Q, K, V, ws_, ex, sa, D, dn, seed=11, layer=0) for ex, sa in ws_.sweep]
+    pts.append(budget_point(ig, Q, K, V, ws_, ws_.exact_frac, 0.0, D, dn, seed=11, layer=0))
+    del Q, K, V, D
+    torch.cuda.empty_cache()
+    return {"workload": ws_.name, "layers_run": 1, "layer": 0, "heads": ws_.B * ws_.H,
+            "note": "one full 40-head layer of the 40-layer stack; the other layers share its shape and recipe",
+            "points": pts}
 
 
 def workload_config(w, exact, sample, selection="centroid"):
@@ -345,7 +411,10 @@ def main():
     # HBM-side stages: algorithmic bytes
     BH, N, d = w.B * w.H, w.N, w.d
     m = ig.sample_budget(p)
-    bytes_cluster = lambda C: w.iters * (BH * N * d * 2 * 2 + BH * N * 4 * 3) + BH * C * d * 4 * 2
+    # k-means: one read of the tokens and one int32 assignment per token per
+    # iteration (the method's algorithmic traffic; the update's second pass
+    # over the tokens is not counted)
+    bytes_cluster = lambda C: w.iters * (BH * N * d * 2 + BH * N * 4)
     hbm = {
         "cluster_q": bytes_cluster(w.Cq), "cluster_k": bytes_cluster(w.Ck),
         "gather_kv": 2 * 2 * BH * N * d * 2 + BH * N * 4,
@@ -356,7 +425,8 @@ def main():
         e = {"ms": round(stage_ms[s], 3)}
         if s in hbm:
             gbs = hbm[s] / (stage_ms[s] * 1e-3) / 1e9
-            e.update(gbs=round(gbs, 1), hbm_frac=round(gbs / peaks["hbm"], 3))
+            e.update(algorithmic_bytes=int(hbm[s]), gbs=round(gbs, 1), hbm_frac=round(gbs / peaks["hbm"], 3),
+                     hbm_peak_gbs=peaks["hbm"])
         stage_report[s] = e
     kmeans_flops = 2 * BH * N * (w.Cq + w.Ck) * d * 2 * w.iters     # hi+lo operand: K = 2d
     stage_report["cluster_q"]["tensor_tflops"] = round(
@@ -387,6 +457,15 @@ def main():
         num = (O.float() - D.float()).pow(2).sum().sqrt()
         den = D.float().pow(2).sum().sqrt()
         extra["rel_l2_vs_dense"] = round(float(num / den), 4)
+        if not args.no_sweeps and not pq:
+            # density ends of the budget range on the same inputs (untimed
+            # for the headline value; each point timed on its own)
+            Df = D.float()
+            dn = float(Df.pow(2).sum().sqrt())
+            extra["density_sweep"] = [budget_point(ig, Q, K, V, w, ex, sa, Df, dn, seed=1000 + rank, layer=rank,
+                                                   ws=ws)
+                                      for ex, sa in ((0.04, 0.04), (0.32, 0.32))]
+            del Df
         del D
 
     # ---------------- end to end through the public API with host buffers
@@ -417,6 +496,10 @@ def main():
                "d2h_bytes_per_step": O.numel() * 2, "steps": ksteps}
         del hQ, hK, hV, hO, hws
 
+    # ---------------- the stack's sample-budget sweep (untimed for the value)
+    if not args.no_dense and not args.no_sweeps and not pq and args.heads is None and w.name == "wan2.1-14b_720p":
+        extra["stack_sample_sweep"] = stack_sample_sweep(ig, dev, args)
+
     # ---------------- max over ranks
     ms_call, value, e2e_value = job_time(t_fwd, e2e["value"] if e2e else 0.0, args.steps, world, dist, dev)
     if e2e:
@@ -424,14 +507,15 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not pq:  # the sample runs the centroid ranking
-        orc = OracleSample(w, exact, sample)
+        orc = OracleSample(w, exact, sample, layer=rank)
         orc.step()
         vals = [orc.step() for _ in range(3)]
         cpu = {"value": round(statistics.median(vals), 1), "unit": "ms/call", "cores": orc.oracle.num_threads(),
-               "kind": "oracle", "sample": orc.describe() + "; median of 3 steps"}
+               "kind": "oracle", "sample": orc.describe() + "; median of 3 steps", **orc.fields()}
 
     launches_per_step = 2 * (1 + 3 * w.iters) + 1 + 1 + 1 + (2 if pq else 0)  # + codebooks, votes
-    peak_sust = peaks["bf16_sust"]
+    peak = peaks["bf16"]  # the burst figure: the kernel is timed per call, not in a seconds-long loop
+    clk_frac = (clocks["sm_mhz"] / clocks["sm_max_mhz"]) if clocks.get("sm_mhz") and clocks.get("sm_max_mhz") else None
     line = {
         "metric": "ms per InstaGen attention call", "value": round(value, 3), "unit": "ms/call",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_call, 3),
@@ -440,11 +524,13 @@ def main():
         "effective_tflops": round(attended_flops / (ms_call * 1e-3) / 1e12, 1),
         "attended_flops": attended_flops, "density": round(density, 4),
         "roofline": {"kernel": "attention", "bound": "tensor", "achieved": round(achieved, 1),
-                     "peak": peak_sust, "unit": "TFLOP/s", "frac": round(achieved / peak_sust, 4),
-                     "peak_kind": f"bf16 sustained ({peaks['source']})",
-                     "frac_of_burst": round(achieved / peaks["bf16"], 4),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_kind": f"bf16 burst ({peaks['source']})",
+                     "frac_clock_matched": (round(achieved / (peak * clk_frac), 4) if clk_frac else None),
+                     "clock_matched_peak": (round(peak * clk_frac, 1) if clk_frac else None),
+                     "frac_of_sustained": round(achieved / peaks["bf16_sust"], 4),
                      "traffic": traffic, "algorithmic_unit": "4*d FLOPs per attended (query,key) pair",
-                     "ms": round(t_att, 3)},
+                     "flops_per_launch": attended_flops, "ms": round(t_att, 3)},
         "stages": stage_report,
         "e2e": ({"value": round(e2e["value"], 3), "unit": "ms/call", "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
                  "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]} if e2e else None),

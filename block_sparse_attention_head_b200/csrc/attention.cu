@@ -8,31 +8,41 @@
 // CTA = two tiles of 128 queries (Q0, Q1) of one query group, gathered from Q
 // through the query permutation.  Both share the group's key list: its exact
 // groups (rank order; contiguous ranges of the permuted K/V) followed by its m
-// sample slots (gathered rows with log-weight w), walked in tiles of 128 keys.
-// Per key tile j and query tile t:
+// sample slots (gathered rows with log-weight w), walked in tiles of 128 keys,
+// so every K/V tile brought on chip serves 256 queries.  Per key tile j and
+// query tile t:
 //   S_t = Q_t K_j^T + 1 w_j^T/scale    tcgen05 (M=128, N=128, bf16), fp32 in
 //                          TMEM: d/16 steps over Q and K plus one side step
 //                          whose 16-column operands hold (1, 1) per query row
 //                          and (w_hi, w_lo) per key slot (w/scale in two bf16
 //                          terms; -inf for padding slots, 0 for exact keys)
-//   P_t = 2^(S_t*scale*log2e - m_t)    softmax warpgroup t, written back as
-//                          fp16 into S_t's TMEM columns
+//   P_t = 2^(S_t*scale*log2e - m_t)    softmax, written back as fp16 into
+//                          S_t's TMEM columns
 //   O_t += P_t V_j         tcgen05 with A (P_t) read from TMEM, fp16 operands
-// Folding w into the product leaves the softmax one code path with no
-// per-column loads.  The tensor pipe alternates [PV_0(j-1), S_0(j)] and
-// [PV_1(j-1), S_1(j)], so one warpgroup's softmax runs while the other tile's
-// MMAs execute.  The running max is only raised when it grows by more than 8
-// (log2 units), so P <= 256 and the O rescale (a TMEM read-modify-write) is
-// rare; it is done by the softmax warpgroup after S_t(j) lands, which the MMA
-// pipe orders after PV_t(j-1).  P and V are fp16 (V converted by the gather):
-// 11 mantissa bits keep the output within 2e-3 mean relative error after its
+// A CTA left with one query tile (a group's odd last tile) runs two chains
+// over that tile instead: chain 0 takes the even key tiles and chain 1 the
+// odd ones, each with its own S buffer, O accumulator and running max, and
+// the epilogue merges the two partial softmaxes; so every CTA keeps two
+// independent S -> softmax -> PV chains in flight.
+// The tensor pipe alternates [PV_0(j-1), S_0(j)] and [PV_1(j-1), S_1(j)].  The
+// softmax is one team of eight warps that takes the tiles in that same order
+// (S_0(j), S_1(j), S_0(j+1), ...): two warps per SM sub-partition share each
+// tile, one thread per half row, so one tile's exponentials run on every
+// MUFU unit at once while the other tile's MMAs execute, and the two tiles'
+// softmaxes never compete for the MUFU.  The two halves of a row agree on
+// its running max through shared memory (one exchange per tile); each keeps
+// its own partial row sum.  The running max is only raised when it grows by
+// more than 8 (log2 units), so P <= 256 and the O rescale (a TMEM
+// read-modify-write) is rare; it runs after S_t(j) lands, which the MMA pipe
+// orders after PV_t(j-1).  P and V are fp16 (V converted by the gather): 11
+// mantissa bits keep the output within 2e-3 mean relative error after its
 // bf16 rounding.
 //
 // Warps: 0 MMA issuer + TMEM owner, 1 idle, 2-3 producer (cp.async 16-byte
 // row gathers into the 128-byte-swizzled operand layout, completion tracked
 // by the stage mbarriers so the producer never blocks on memory; the key side
-// rows are plain shared stores), 4-7 softmax for Q0, 8-11 softmax for Q1
-// (thread = query row = TMEM lane).
+// rows are plain shared stores), 4-11 softmax: warp w owns TMEM lane quarter
+// w mod 4 (query rows 32(w mod 4) + lane) and column half (w - 4) / 4.
 #include "internal.cuh"
 #include "ptx.cuh"
 
@@ -44,6 +54,7 @@ namespace ig {
 namespace {
 constexpr int kAttnThreads = 384;
 constexpr int kProducers = 64;
+constexpr int kSoftmaxThreads = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;
 
@@ -60,12 +71,15 @@ struct AttnSmem {
   static constexpr int kKx = kQx + kSideBytes;                // 2 stages
   static constexpr int kGStart = kKx + 2 * kSideBytes;        // exact group start slots
   static constexpr int kGPre = kGStart + kAttnMaxExactGroups * 4;  // exclusive prefix of sizes
-  static constexpr int kBars = (kGPre + (kAttnMaxExactGroups + 1) * 4 + 15) / 16 * 16;
+  // half-row exchange: [2 slots][2 halves][128 rows] fp32
+  static constexpr int kXch = (kGPre + (kAttnMaxExactGroups + 1) * 4 + 15) / 16 * 16;
+  static constexpr int kBars = kXch + 2 * 2 * 128 * 4;
   static constexpr int kNumBars = 16;
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kBytes = kMisc + 64;
-  static size_t bytes() { return 1024 + kBytes; }
+  static constexpr size_t bytes() { return 1024 + kBytes; }
 };
+static_assert(AttnSmem<128>::bytes() <= 232448, "shared memory budget");
 
 template <typename T>
 __device__ __forceinline__ const T* row_ptr(const T* base, int bh, int N, int row, int D) {
@@ -81,6 +95,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   int* gstart = reinterpret_cast<int*>(smem + L::kGStart);
   int* gpre = reinterpret_cast<int*>(smem + L::kGPre);
+  float* xch = reinterpret_cast<float*>(smem + L::kXch);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;   // [2] stages
@@ -138,6 +153,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
   const int rows0 = min(128, qhi - q0);
   const int rows1 = max(0, min(128, qhi - q0 - 128));
   const int ntiles = rows1 > 0 ? 2 : 1;
+  // one query tile: chains 0 and 1 split the key tiles (even / odd) of tile 0
+  const bool split = ntiles == 1;
   const int n_exact = a.counts[grp * 3 + 0];
   const int ns = a.counts[grp * 3 + 2];
   if (qlo < 0 || qhi > N || rows0 < 1 || n_exact < 1 || n_exact > Ck || n_exact > kAttnMaxExactGroups || ns < 0 ||
@@ -186,7 +203,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
       mbar_init(&k_empty[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+      mbar_init(&p_full[s], kSoftmaxThreads);
     }
     mbar_init(o_done, 1);
     mbar_init(fin, 1);
@@ -335,173 +352,248 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
         wA = slot_w(kt + 1, rA);
         wB = slot_w(kt + 1, rB);
       }
-      if (kt >= 2 && !mbar_wait(&k_empty[s], (use - 1) & 1, abort_flag)) break;
+      // warp-uniform waits: every lane reaches the shuffles below together
+      if (kt >= 2 && !mbar_wait_warp(&k_empty[s], (use - 1) & 1, abort_flag)) break;
       side_row(kx_s + s * L::kSideBytes, rA, cwA);
       side_row(kx_s + s * L::kSideBytes, rB, cwB);
       fence_proxy_async_smem();
       mbar_arrive(&k_full[s]);
       issue_rows(a.Kp, k_s + s * L::kTileBytes, posA, posB);
       cp_async_arrive_noinc(&k_full[s]);
-      if (kt >= 2 && !mbar_wait(&v_empty[s], (use - 1) & 1, abort_flag)) break;
+      if (kt >= 2 && !mbar_wait_warp(&v_empty[s], (use - 1) & 1, abort_flag)) break;
       issue_rows(a.Vp, v_s + s * L::kTileBytes, posA, posB);
       cp_async_arrive_noinc(&v_full[s]);
     }
     cp_async_wait_all();
   } else if (warp >= 4) {
     // ================================================================= softmax
-    const int t = (warp - 4) >> 2;          // query tile of this warpgroup
-    const int r = tid - 128 - 128 * t;      // query row == TMEM lane
-    const uint32_t lane_off = (uint32_t)((r & ~31) << 16);
-    const uint32_t s_col = tmem + lane_off + (uint32_t)(128 * t);
-    const uint32_t o_col = tmem + lane_off + (uint32_t)(256 + 128 * t);
-    const bool active = t < ntiles;
-    float m_run = -__int_as_float(0x7f800000);
-    float l_run = 0.f;
-    bool ok = active;
+    const int qd = warp & 3;               // TMEM lane quarter
+    const int hf = (warp - 4) >> 2;        // column half of S and O
+    const int r = 32 * qd + lane;          // query row == TMEM lane
+    const uint32_t lane_off = (uint32_t)((32 * qd) << 16);
+    float m_run[2], l_run[2];
+    m_run[0] = m_run[1] = -__int_as_float(0x7f800000);
+    l_run[0] = l_run[1] = 0.f;
+    bool ok = true;
+    int xs = 0;  // exchange slot, alternating per tile visit
     for (int kt = 0; kt < ntk && ok; ++kt) {
-      if (!mbar_wait_warp(&s_full[t], kt & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // the whole S row of this thread in registers: one TMEM round trip; S
-      // already carries the column log-weights (side step of the product)
-      float x[128];
-      tmem_ld32(s_col + 0, x);
-      tmem_ld32(s_col + 32, x + 32);
-      tmem_ld32(s_col + 64, x + 64);
-      tmem_ld32(s_col + 96, x + 96);
-      tmem_wait_ld();
-      float mxp[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) mxp[e] = -__int_as_float(0x7f800000);
-#pragma unroll
-      for (int c = 0; c < 128; c += 2) mxp[(c >> 1) & 3] = fmax3(mxp[(c >> 1) & 3], x[c], x[c + 1]);
-      // scale after the max (scale > 0)
-      const float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])) * a.scale_log2;
-      const float m_new = fmaxf(m_run, mx);
-      const bool rescale = m_new > m_run + kRescaleThreshold;
-      float alpha = 1.f;
-      if (rescale) {
-        alpha = ex2_approx(m_run - m_new);
-        m_run = m_new;
-      }
-      // P = 2^(x - m) as fp16 pairs into the first 64 columns of S_t (already
-      // read); the pairs are packed in place into slots of x already consumed
-      const float neg_m = -m_run;
-      float rsp[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int c = c4 * 32 + e;
-          const float p0 = ex2_approx(fmaf(x[c], a.scale_log2, neg_m));
-          const float p1 = ex2_approx(fmaf(x[c + 1], a.scale_log2, neg_m));
-          rsp[(e >> 1) & 3] += p0 + p1;
-          x[c4 * 16 + (e >> 1)] = __uint_as_float(pack_f16x2(p0, p1));
+      for (int t = 0; t < 2; ++t) {
+        // chain t handles key tile kt (split: only the chain of kt's parity)
+        if (split ? (kt & 1) != t : t >= ntiles) continue;
+        const int ph = split ? (kt >> 1) : kt;       // visit index of chain t
+        const bool first = ph == 0;                  // the chain's first key tile
+        const uint32_t s_col = tmem + lane_off + (uint32_t)(128 * t + 64 * hf);
+        const uint32_t o_col = tmem + lane_off + (uint32_t)(256 + 128 * t + (D / 2) * hf);
+        if (!mbar_wait_warp(&s_full[t], ph & 1, abort_flag)) {
+          ok = false;
+          break;
         }
-        tmem_st16(s_col + c4 * 16, reinterpret_cast<const uint32_t*>(x + c4 * 16));
-      }
-      const float rs = (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
-      // O_t holds PV_t(kt-1) (the MMA pipe ran it before S_t(kt)) and PV_t(kt)
-      // waits for p_full; tcgen05.ld/st are warp-collective, so the warp
-      // rescales if any of its rows needs it (done after P so x is dead here)
-      if (kt >= 1 && __any_sync(0xffffffffu, rescale)) {
+        tc_fence_after();
+        // this thread's half row of S: 64 columns, one TMEM round trip; S
+        // already carries the column log-weights (side step of the product)
+        float x[64];
+        tmem_ld32(s_col + 0, x);
+        tmem_ld32(s_col + 32, x + 32);
+        tmem_wait_ld();
+        float mxp[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mxp[e] = -__int_as_float(0x7f800000);
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) mxp[(c >> 1) & 3] = fmax3(mxp[(c >> 1) & 3], x[c], x[c + 1]);
+        // The two halves of the row exchange their maxima.  Slots alternate
+        // per visit: a slot is rewritten two visits later, after the partner
+        // has passed the barrier of the visit in between, so after its read.
+        const float hmax = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
+        float* slot = xch + xs * 256;
+        slot[hf * 128 + r] = hmax;
+        named_bar_sync(1 + qd, 64);
+        const float omax = slot[(hf ^ 1) * 128 + r];
+        xs ^= 1;
+        // scale after the max (scale > 0)
+        const float mx = fmaxf(hmax, omax) * a.scale_log2;
+        const float m_new = fmaxf(m_run[t], mx);
+        const bool rescale = m_new > m_run[t] + kRescaleThreshold;
+        float alpha = 1.f;
+        if (rescale) {
+          alpha = ex2_approx(m_run[t] - m_new);
+          m_run[t] = m_new;
+        }
+        // P = 2^(x - m) as fp16 pairs: key 64hf + c -> P column 64hf + c/2, in
+        // the first half of this half's own S columns (already read), packed
+        // in place into slots of x already consumed
+        const float neg_m = -m_run[t];
+        float rsp[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t p_col = s_col;
+#pragma unroll
+        for (int c4 = 0; c4 < 2; ++c4) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int c = c4 * 32 + e;
+            const float p0 = ex2_approx(fmaf(x[c], a.scale_log2, neg_m));
+            const float p1 = ex2_approx(fmaf(x[c + 1], a.scale_log2, neg_m));
+            rsp[(e >> 1) & 3] += p0 + p1;
+            x[c4 * 16 + (e >> 1)] = __uint_as_float(pack_f16x2(p0, p1));
+          }
+          tmem_st16(p_col + c4 * 16, reinterpret_cast<const uint32_t*>(x + c4 * 16));
+        }
+        const float rs = (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
+        // O_t holds the chain's earlier PVs (the MMA pipe ran them before
+        // S_t(kt)) and the next one waits for p_full; tcgen05.ld/st are
+        // warp-collective, so the warp rescales its half of O if any of its
+        // rows needs it
+        if (!first && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
-        for (int c4 = 0; c4 < D / 32; ++c4) {
-          float o[32];
-          tmem_ld32(o_col + c4 * 32, o);
-          tmem_wait_ld();
+          for (int c4 = 0; c4 < D / 64; ++c4) {
+            float o[32];
+            tmem_ld32(o_col + c4 * 32, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tmem_st32(o_col + c4 * 32, o);
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tmem_st32(o_col + c4 * 32, o);
+          }
         }
+        tmem_wait_st();
+        l_run[t] = l_run[t] * alpha + rs;
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
       }
-      tmem_wait_st();
-      l_run = l_run * alpha + rs;
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
     }
     if (ok && mbar_wait_warp(o_done, 0, abort_flag)) {
       tc_fence_after();
-      const float inv = 1.f / l_run;
-      const int nrows = t == 0 ? rows0 : rows1;
-      bool valid = r < nrows;
-      int tok = 0;
-      if (valid) {
-        tok = a.q_perm[(size_t)bh * N + q0 + 128 * t + r];
-        if (tok < 0 || tok >= N) valid = false;
+      // row sums: the two halves' partial sums.  Every softmax thread has
+      // arrived on p_full of its last tile before o_done, so each has read
+      // the partner's last maximum and the whole exchange area is free.
+      xch[hf * 128 + r] = l_run[0];
+      xch[256 + hf * 128 + r] = l_run[1];
+      named_bar_sync(1 + qd, 64);
+      float lsum[2] = {l_run[0] + xch[(hf ^ 1) * 128 + r], l_run[1] + xch[256 + (hf ^ 1) * 128 + r]};
+      // split: the two chains' partial softmaxes of the same rows merge with
+      // weights 2^(m_c - max(m_0, m_1)); chain 1 is empty when ntk == 1
+      float wgt[2] = {1.f, 1.f};
+      const bool two = split && ntk > 1;
+      if (two) {
+        const float mm = fmaxf(m_run[0], m_run[1]);
+        wgt[0] = ex2_approx(m_run[0] - mm);
+        wgt[1] = ex2_approx(m_run[1] - mm);
+        lsum[0] = lsum[0] * wgt[0] + lsum[1] * wgt[1];
       }
-      __nv_bfloat16* dst = a.O + ((size_t)bh * N + tok) * D;
-#pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) {
-        float o[32];
-        tmem_ld32(o_col + c4 * 32, o);
-        tmem_wait_ld();
+      for (int t = 0; t < ntiles; ++t) {
+        const float inv = 1.f / lsum[t];
+        const uint32_t o_col = tmem + lane_off + (uint32_t)(256 + 128 * t + (D / 2) * hf);
+        const int nrows = t == 0 ? rows0 : rows1;
+        bool valid = r < nrows;
+        int tok = 0;
         if (valid) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c4 * 32);
+          tok = a.q_perm[(size_t)bh * N + q0 + 128 * t + r];
+          if (tok < 0 || tok >= N) valid = false;
+        }
+        __nv_bfloat16* dst = a.O + ((size_t)bh * N + tok) * D + (D / 2) * hf;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            d4[q] = make_uint4(pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv),
-                               pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
-                               pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
-                               pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+        for (int c4 = 0; c4 < D / 64; ++c4) {
+          float o[32];
+          tmem_ld32(o_col + c4 * 32, o);
+          tmem_wait_ld();
+          if (two) {
+            float o1[32];
+            tmem_ld32(o_col + 128 + c4 * 32, o1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = o[e] * wgt[0] + o1[e] * wgt[1];
+          }
+          if (valid) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c4 * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              d4[q] = make_uint4(pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv),
+                                 pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                 pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                 pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+            }
           }
         }
       }
     }
   } else if (warp == 0 && lane == 0) {
     // ===================================================================== MMA
+    // Descriptors are formed once and advanced by adding (byte offset >> 4)
+    // to their start-address field, so the issue loop is little more than
+    // the MMA instructions themselves.
     const uint32_t idesc_qk = umma_idesc_bf16(128, 128, false, false);
     const uint32_t idesc_pv = umma_idesc_f16kind(128, D, false, true, true);  // fp16 P (TMEM) x fp16 V
+    const uint64_t qd0 = umma_desc_sw128(q_s, 16, 1024);
+    const uint64_t kd0 = umma_desc_sw128(k_s, 16, 1024);
+    const uint64_t vd0 = umma_desc_sw128(v_s, 16384, 1024);
+    const uint64_t qxd = umma_desc_noswz(qx_s, 128, 256);
+    const uint64_t kxd0 = umma_desc_noswz(kx_s, 128, 256);
+    constexpr uint64_t kTileStep = (uint64_t)(L::kTileBytes >> 4);
+    constexpr uint64_t kSideStep = (uint64_t)(L::kSideBytes >> 4);
     bool ok = mbar_wait(q_full, 0, abort_flag);
     fence_proxy_async_smem();
-    // O_t += P_t(j) V(j), A operand = P_t in TMEM (columns of S_t)
-    auto issue_pv = [&](int t, int j) -> bool {
-      if (!mbar_wait(&p_full[t], j & 1, abort_flag)) return false;
-      tc_fence_after();
-      const uint32_t vb = v_s + (j & 1) * L::kTileBytes;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint64_t bd = umma_desc_sw128(vb + k * 2048, 16384, 1024);
-        umma_f16_ts(tmem + 256 + 128 * t, tmem + 128 * t + 8 * k, bd, idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
-      }
-      return true;
-    };
+    // Per key tile kt and chain t: PV_t(kt-1), then S_t(kt).  Each wait sits
+    // right before the first MMA that needs it, so a chain whose P is ready
+    // never waits for the next K tile's copies.  Split: chain t only has the
+    // key tiles of its parity, so a key tile's S comes before the other
+    // chain's PV of the previous one.
     for (int kt = 0; kt <= ntk && ok; ++kt) {
-      const int s = kt & 1;
-      if (kt < ntk) {
-        if (!mbar_wait(&k_full[s], (kt >> 1) & 1, abort_flag)) break;
-        fence_proxy_async_smem();
-      }
-      if (kt >= 1) {
-        if (!mbar_wait(&v_full[(kt - 1) & 1], ((kt - 1) >> 1) & 1, abort_flag)) break;
-        fence_proxy_async_smem();
-      }
-      tc_fence_after();
-      for (int t = 0; t < ntiles && ok; ++t) {
-        if (kt >= 1) {
-          if (!issue_pv(t, kt - 1)) {
+      bool v_waited = false, k_waited = false;
+      for (int u = 0; u < 2 && ok; ++u) {
+        // normal: chain t = u; split: the chain of kt (its S) goes first
+        const int t = split ? ((kt + u) & 1) : u;
+        const int j = kt - 1;  // key tile of the PV
+        const bool pv = j >= 0 && (split ? (j & 1) == t : t < ntiles);
+        const bool sv = kt < ntk && (split ? (kt & 1) == t : t < ntiles);
+        if (pv) {
+          if (!v_waited) {
+            if (!mbar_wait(&v_full[j & 1], (j >> 1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            fence_proxy_async_smem();
+            v_waited = true;
+          }
+          // O_t += P_t(j) V(j), A operand = P_t in TMEM (columns of S_t)
+          const int ph = split ? (j >> 1) : j;
+          if (!mbar_wait(&p_full[t], ph & 1, abort_flag)) {
             ok = false;
             break;
           }
-          if (t == ntiles - 1) umma_commit(&v_empty[(kt - 1) & 1]);
+          tc_fence_after();
+          const uint64_t vd = vd0 + (uint64_t)(j & 1) * kTileStep;
+          const uint32_t o_t = tmem + 256 + 128 * t, p_t = tmem + 128 * t;
+          // keys 16k..16k+15 of P: half k/4 of the tile, whose P occupies the
+          // first 32 columns of that half's S columns
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            umma_f16_ts(o_t, p_t + 8 * k + 32 * (k >> 2), vd + (uint64_t)(k * 128), idesc_pv,
+                        (ph > 0 || k > 0) ? 1u : 0u);
+          // the last PV of key tile j frees its V stage
+          if (split || t == ntiles - 1) umma_commit(&v_empty[j & 1]);
         }
-        if (kt < ntk) {
-          const uint32_t kb = k_s + s * L::kTileBytes;
-          const uint32_t qb = q_s + t * L::kTileBytes;
+        if (sv) {
+          if (!k_waited) {
+            if (!mbar_wait(&k_full[kt & 1], (kt >> 1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            fence_proxy_async_smem();
+            tc_fence_after();
+            k_waited = true;
+          }
+          const uint64_t kd = kd0 + (uint64_t)(kt & 1) * kTileStep;
+          const uint64_t kxd = kxd0 + (uint64_t)(kt & 1) * kSideStep;
+          const uint64_t qd = qd0 + (uint64_t)(split ? 0 : t) * kTileStep;
+          const uint32_t s_t = tmem + 128 * t;
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
-            const uint64_t ad = umma_desc_sw128(qb + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-            const uint64_t bd = umma_desc_sw128(kb + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-            umma_bf16_ss(tmem + 128 * t, ad, bd, idesc_qk, k > 0 ? 1u : 0u);
+            const uint64_t off = (uint64_t)((k >> 2) * 1024 + (k & 3) * 2);
+            umma_bf16_ss(s_t, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
           }
-          umma_bf16_ss(tmem + 128 * t, umma_desc_noswz(qx_s, 128, 256),
-                       umma_desc_noswz(kx_s + s * L::kSideBytes, 128, 256), idesc_qk, 1u);
+          umma_bf16_ss(s_t, qxd, kxd, idesc_qk, 1u);
           umma_commit(&s_full[t]);
+          // the last S of key tile kt frees its K stage
+          if (split || t == ntiles - 1) umma_commit(&k_empty[kt & 1]);
         }
       }
-      if (ok && kt < ntk) umma_commit(&k_empty[s]);
     }
     if (ok) umma_commit(o_done);
     umma_commit(fin);

@@ -351,6 +351,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       : "memory");
 }
 
+// 8 consecutive 32-bit columns of this thread's TMEM lane: `first`, then
+// seven copies of `rest`.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, uint32_t first, uint32_t rest) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%2,%2,%2,%2,%2,%2};" ::"r"(taddr), "r"(first),
+               "r"(rest)
+               : "memory");
+}
+
 // 16 consecutive 32-bit columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile(
