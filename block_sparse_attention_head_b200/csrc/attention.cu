@@ -38,7 +38,11 @@
 // mantissa bits keep the output within 2e-3 mean relative error after its
 // bf16 rounding.
 //
-// Warps: 0 MMA issuer + TMEM owner, 1 idle, 2-3 producer (cp.async 16-byte
+// Warps: 0 TMEM owner and MMA warp of chain 0, 1 MMA warp of chain 1 (each
+// chain's MMAs come from one elected lane, in order; two issuers keep the
+// tensor pipe fed while either one waits on a barrier or sits in the issue of
+// an MMA instruction, which takes about as long as the MMA itself), 2-3
+// producer (cp.async 16-byte
 // row gathers into the 128-byte-swizzled operand layout, completion tracked
 // by the stage mbarriers so the producer never blocks on memory; the key side
 // rows are plain shared stores), 4-11 softmax: warp w owns TMEM lane quarter
@@ -200,13 +204,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 2 * kProducers);
       mbar_init(&v_full[s], kProducers);
-      mbar_init(&k_empty[s], 1);
-      mbar_init(&v_empty[s], 1);
+      // a key tile's K and V stages are freed by every chain that reads them
+      mbar_init(&k_empty[s], split ? 1 : 2);
+      mbar_init(&v_empty[s], split ? 1 : 2);
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], kSoftmaxThreads);
     }
-    mbar_init(o_done, 1);
-    mbar_init(fin, 1);
+    mbar_init(o_done, 2);  // one commit per chain
+    mbar_init(fin, 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -513,11 +518,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
         }
       }
     }
-  } else if (warp == 0 && lane == 0) {
+  } else if (warp < 2) {
     // ===================================================================== MMA
+    // Warp t issues chain t: S_t(j0), then for each further key tile j of the
+    // chain PV_t(previous), S_t(j), and finally PV_t(last).  The whole warp
+    // runs the loop and its waits in step (so descriptors and loop state are
+    // warp-uniform) and one elected lane issues the MMAs and commits.
     // Descriptors are formed once and advanced by adding (byte offset >> 4)
-    // to their start-address field, so the issue loop is little more than
-    // the MMA instructions themselves.
+    // to their start-address field; each wait sits right before the first
+    // MMA that needs it.
+    const int t = warp;
     const uint32_t idesc_qk = umma_idesc_bf16(128, 128, false, false);
     const uint32_t idesc_pv = umma_idesc_f16kind(128, D, false, true, true);  // fp16 P (TMEM) x fp16 V
     const uint64_t qd0 = umma_desc_sw128(q_s, 16, 1024);
@@ -527,76 +537,72 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
     const uint64_t kxd0 = umma_desc_noswz(kx_s, 128, 256);
     constexpr uint64_t kTileStep = (uint64_t)(L::kTileBytes >> 4);
     constexpr uint64_t kSideStep = (uint64_t)(L::kSideBytes >> 4);
-    bool ok = mbar_wait(q_full, 0, abort_flag);
+    const uint64_t qd = qd0 + (uint64_t)(split ? 0 : t) * kTileStep;
+    const uint32_t s_t = tmem + 128 * t, o_t = tmem + 256 + 128 * t;
+    // chain t's key tiles: all of them, or (split) those of parity t
+    const bool active = split || t < ntiles;
+    const int j0 = split ? t : 0, jstep = split ? 2 : 1;
+    bool ok = mbar_wait_warp(q_full, 0, abort_flag);
     fence_proxy_async_smem();
-    // Per key tile kt and chain t: PV_t(kt-1), then S_t(kt).  Each wait sits
-    // right before the first MMA that needs it, so a chain whose P is ready
-    // never waits for the next K tile's copies.  Split: chain t only has the
-    // key tiles of its parity, so a key tile's S comes before the other
-    // chain's PV of the previous one.
-    for (int kt = 0; kt <= ntk && ok; ++kt) {
-      bool v_waited = false, k_waited = false;
-      for (int u = 0; u < 2 && ok; ++u) {
-        // normal: chain t = u; split: the chain of kt (its S) goes first
-        const int t = split ? ((kt + u) & 1) : u;
-        const int j = kt - 1;  // key tile of the PV
-        const bool pv = j >= 0 && (split ? (j & 1) == t : t < ntiles);
-        const bool sv = kt < ntk && (split ? (kt & 1) == t : t < ntiles);
-        if (pv) {
-          if (!v_waited) {
-            if (!mbar_wait(&v_full[j & 1], (j >> 1) & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            fence_proxy_async_smem();
-            v_waited = true;
-          }
-          // O_t += P_t(j) V(j), A operand = P_t in TMEM (columns of S_t)
-          const int ph = split ? (j >> 1) : j;
-          if (!mbar_wait(&p_full[t], ph & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t vd = vd0 + (uint64_t)(j & 1) * kTileStep;
-          const uint32_t o_t = tmem + 256 + 128 * t, p_t = tmem + 128 * t;
-          // keys 16k..16k+15 of P: half k/4 of the tile, whose P occupies the
-          // first 32 columns of that half's S columns
+    // O_t += P_t(j) V(j), A operand = P_t in TMEM (columns of S_t); keys
+    // 16k..16k+15 of P sit in half k/4 of the tile, whose P occupies the
+    // first 32 columns of that half's S columns
+    auto issue_pv = [&](int j) -> bool {
+      if (!mbar_wait_warp(&v_full[j & 1], (j >> 1) & 1, abort_flag)) return false;
+      const int ph = split ? (j >> 1) : j;
+      if (!mbar_wait_warp(&p_full[t], ph & 1, abort_flag)) return false;
+      fence_proxy_async_smem();
+      tc_fence_after();
+      const uint64_t vd = vd0 + (uint64_t)(j & 1) * kTileStep;
+      if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            umma_f16_ts(o_t, p_t + 8 * k + 32 * (k >> 2), vd + (uint64_t)(k * 128), idesc_pv,
-                        (ph > 0 || k > 0) ? 1u : 0u);
-          // the last PV of key tile j frees its V stage
-          if (split || t == ntiles - 1) umma_commit(&v_empty[j & 1]);
-        }
-        if (sv) {
-          if (!k_waited) {
-            if (!mbar_wait(&k_full[kt & 1], (kt >> 1) & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            fence_proxy_async_smem();
-            tc_fence_after();
-            k_waited = true;
-          }
-          const uint64_t kd = kd0 + (uint64_t)(kt & 1) * kTileStep;
-          const uint64_t kxd = kxd0 + (uint64_t)(kt & 1) * kSideStep;
-          const uint64_t qd = qd0 + (uint64_t)(split ? 0 : t) * kTileStep;
-          const uint32_t s_t = tmem + 128 * t;
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint64_t off = (uint64_t)((k >> 2) * 1024 + (k & 3) * 2);
-            umma_bf16_ss(s_t, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
-          }
-          umma_bf16_ss(s_t, qxd, kxd, idesc_qk, 1u);
-          umma_commit(&s_full[t]);
-          // the last S of key tile kt frees its K stage
-          if (split || t == ntiles - 1) umma_commit(&k_empty[kt & 1]);
-        }
+        for (int k = 0; k < 8; ++k)
+          umma_f16_ts(o_t, s_t + 8 * k + 32 * (k >> 2), vd + (uint64_t)(k * 128), idesc_pv,
+                      (ph > 0 || k > 0) ? 1u : 0u);
+        umma_commit(&v_empty[j & 1]);
       }
+      __syncwarp();
+      return true;
+    };
+    auto issue_s = [&](int j) -> bool {
+      if (!mbar_wait_warp(&k_full[j & 1], (j >> 1) & 1, abort_flag)) return false;
+      fence_proxy_async_smem();
+      tc_fence_after();
+      const uint64_t kd = kd0 + (uint64_t)(j & 1) * kTileStep;
+      const uint64_t kxd = kxd0 + (uint64_t)(j & 1) * kSideStep;
+      if (elect_one()) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t off = (uint64_t)((k >> 2) * 1024 + (k & 3) * 2);
+          umma_bf16_ss(s_t, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
+        }
+        umma_bf16_ss(s_t, qxd, kxd, idesc_qk, 1u);
+        umma_commit(&s_full[t]);
+        umma_commit(&k_empty[j & 1]);
+      }
+      __syncwarp();
+      return true;
+    };
+    if (active) {
+      int prev = -1;
+      for (int j = j0; j < ntk && ok; j += jstep) {
+        if (prev >= 0 && !issue_pv(prev)) {
+          ok = false;
+          break;
+        }
+        if (!issue_s(j)) {
+          ok = false;
+          break;
+        }
+        prev = j;
+      }
+      if (ok && prev >= 0) ok = issue_pv(prev);
     }
-    if (ok) umma_commit(o_done);
-    umma_commit(fin);
+    if (elect_one()) {
+      if (ok) umma_commit(o_done);
+      umma_commit(fin);
+    }
+    __syncwarp();
     mbar_wait_drain(fin, 0);
   }
   tc_fence_before();
