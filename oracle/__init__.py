@@ -76,6 +76,10 @@ def _load():
     lib.orc_select_sample_group.restype = i32
     lib.orc_select_sample.argtypes = [P, i32, P, i32, i32, f32, P, ctypes.POINTER(_SelectCfg), P,
                                       P, P, P, P]
+    lib.orc_select_top_p_group.argtypes = [P, P, i32, f32, i64, P, P, P, P]
+    lib.orc_select_top_p_group.restype = i32
+    lib.orc_select_top_p.argtypes = [P, i32, P, i32, i32, f32, P, f32, i64, P, P]
+    lib.orc_select_top_p.restype = i32
     lib.orc_pq_codebook.argtypes = [P, i32, i32, P, P]
     lib.orc_pq_codebook.restype = i32
     lib.orc_pq_encode.argtypes = [P, i64, i32, P, i32, P]
@@ -256,6 +260,37 @@ def select_sample(cq, ck, k_offsets, scale, E, m, seed=0, layer=0, bh=0, mode=IM
     return ex, cnt, pos[:, :m], bias[:, :m]
 
 
+def select_top_p_group(S_row, k_offsets, top_p, floor_keys):
+    """Top-p selection for one query group: dict with the kept groups (rank
+    order), kept keys, the masses W_j and their total T (no draws)."""
+    lib = _load()
+    S_row, koff = _f32(S_row), _i32(k_offsets)
+    Ck = S_row.shape[0]
+    ex = np.empty(Ck, np.int32)
+    cnt = np.empty(3, np.int32)
+    W = np.zeros(Ck, np.uint64)
+    tot = ctypes.c_uint64(0)
+    _check(lib.orc_select_top_p_group(_ptr(S_row), _ptr(koff), Ck, float(np.float32(top_p)), int(floor_keys),
+                                      _ptr(ex), _ptr(cnt), _ptr(W), ctypes.byref(tot)), "select_top_p_group")
+    ne = int(cnt[0])
+    return dict(exact_groups=ex[:ne].copy(), n_exact=ne, exact_keys=int(cnt[1]), n_sample=int(cnt[2]), W=W,
+                total=int(tot.value))
+
+
+def select_top_p(cq, ck, k_offsets, scale, top_p, floor_keys):
+    """Whole head, top-p selection: (exact_groups [Cq,Ck], counts [Cq,3],
+    sample_pos [Cq,0], sample_bias [Cq,0])."""
+    lib = _load()
+    cq, ck, koff = _f32(cq), _f32(ck), _i32(k_offsets)
+    Cq, d = cq.shape
+    Ck = ck.shape[0]
+    ex = np.empty((Cq, Ck), np.int32)
+    cnt = np.empty((Cq, 3), np.int32)
+    _check(lib.orc_select_top_p(_ptr(cq), Cq, _ptr(ck), Ck, d, float(np.float32(scale)), _ptr(koff),
+                                float(np.float32(top_p)), int(floor_keys), _ptr(ex), _ptr(cnt)), "select_top_p")
+    return ex, cnt, np.zeros((Cq, 0), np.int32), np.zeros((Cq, 0), np.float64)
+
+
 # ------------------------------------------------------------ PQ voting (readings
 # in the C source: 8-dimension subspaces, 16 codewords, 5 Lloyd iterations on
 # the group centroids, per-query budget prefix, votes then centroid score)
@@ -344,11 +379,14 @@ class HeadResult:
 
 
 def forward_head(Q, K, V, *, Cq, Ck, iters, exact_frac, sample_frac, scale, seed=0, layer=0, bh=0,
-                 mode=IMPORTANCE, rows=None, cq_init=None, ck_init=None, selection="centroid") -> HeadResult:
+                 mode=IMPORTANCE, rows=None, cq_init=None, ck_init=None, selection="centroid",
+                 top_p=0.9, key_floor=0.1) -> HeadResult:
     """All stages for one head, in the pages' order.  ``rows`` limits the
     attention stage to those original query indices (all when None).
-    ``selection``: "centroid" (Figure 3) or "pq_vote" (the abstract's
-    product-quantised per-query voting)."""
+    ``selection``: "centroid" (Figure 3), "pq_vote" (the abstract's
+    product-quantised per-query voting) or "top_p" (the SVG2-style comparator:
+    the groups holding the share ``top_p`` of the estimated mass, at least
+    ``key_floor`` of the keys, no sample; exact_frac and sample_frac unused)."""
     Q, K, V = _f32(Q), _f32(K), _f32(V)
     N = Q.shape[0]
     cq, qa, _ = kmeans(Q, Cq, iters, cq_init)
@@ -356,8 +394,11 @@ def forward_head(Q, K, V, *, Cq, Ck, iters, exact_frac, sample_frac, scale, seed
     qp, qo = permutation(qa, Cq)
     kp, ko = permutation(ka, Ck)
     E, m = budget(exact_frac, N), budget(sample_frac, N)
-    votes = pq_votes(Q, cq, ck, qp, qo, ko, E) if selection == "pq_vote" else None
-    ex, cnt, sp, sb = select_sample(cq, ck, ko, scale, E, m, seed, layer, bh, mode, votes)
+    if selection == "top_p":
+        ex, cnt, sp, sb = select_top_p(cq, ck, ko, scale, top_p, budget(key_floor, N))
+    else:
+        votes = pq_votes(Q, cq, ck, qp, qo, ko, E) if selection == "pq_vote" else None
+        ex, cnt, sp, sb = select_sample(cq, ck, ko, scale, E, m, seed, layer, bh, mode, votes)
     if rows is None:
         rows = np.arange(N)
     out = attention_rows(Q, K, V, scale, qa, kp, ko, ex, cnt, sp, sb, rows) if len(rows) else None

@@ -415,6 +415,100 @@ int orc_select_sample(const float* cq, int Cq, const float* ck, int Ck, int d, f
 }
 
 /* ------------------------------------------------------------------------- */
+/* Top-p key-group selection: the comparator the pages set InstaGen against
+ * (thelatestinai.com paper page, Figure 2 caption: SVG2 with Cq = 100,
+ * Ck = 500, key floor 0.1, at top-p 0.5 / 0.75 / 0.9 / 0.95; ICLR listing
+ * abstract: top-p keeps the highest-scoring blocks and varies their number to
+ * reach a target share of the attention mass; the dropped blocks are simply
+ * skipped, with no sample).  Every step beyond that sentence is a [reading]:
+ *   - estimated attention mass of key group j for query group i: |K_j| times
+ *     the per-key estimate exp(S_ij), in the same integer fixed point as the
+ *     sampling weights: W_j = |K_j| * q_j with q_j = orc_group_weight(S_ij,
+ *     max over all non-empty groups of S_ij), T = sum_j W_j;
+ *   - groups ranked by W_j descending (ties: lowest j), the nucleus order;
+ *   - the kept set is the shortest prefix of that ranking whose mass reaches
+ *     the share p, cum * 2^20 >= p_fix * T with p_fix = round(p * 2^20), and
+ *     which holds at least F = round(key_floor * N) keys (the key floor); the
+ *     first-ranked group is always kept;
+ *   - no draws.
+ * Integer arithmetic throughout (T < 2^44 for N < 2^20), so the kept set is
+ * reproducible bit for bit.
+ * Outputs as orc_select_sample_group: exact_groups in rank order (rest -1),
+ * counts = {kept groups, kept keys, 0}; W_out[j] (optional) the masses.      */
+/* ------------------------------------------------------------------------- */
+int orc_select_top_p_group(const float* S_row, const int32_t* k_offsets, int Ck, float top_p,
+                           int64_t floor_keys, int32_t* exact_groups, int32_t* counts,
+                           uint64_t* W_out /* [Ck] or NULL */, uint64_t* total_out /* or NULL */)
+{
+    int32_t* order = (int32_t*)malloc(sizeof(int32_t) * (size_t)(Ck > 0 ? Ck : 1));
+    uint64_t* W = (uint64_t*)calloc((size_t)(Ck > 0 ? Ck : 1), sizeof(uint64_t));
+    if (!order || !W) { free(order); free(W); return ORC_ERR_NOMEM; }
+    const int64_t p_fix = llround((double)top_p * 1048576.0);
+
+    float smax = -INFINITY;
+    int any = 0;
+    for (int j = 0; j < Ck; ++j) {
+        if (k_offsets[j + 1] - k_offsets[j] <= 0) continue;
+        if (!any || S_row[j] > smax) smax = S_row[j];
+        any = 1;
+    }
+    uint64_t total = 0;
+    for (int j = 0; j < Ck; ++j) {
+        const int64_t cnt = k_offsets[j + 1] - k_offsets[j];
+        if (cnt <= 0) continue;
+        W[j] = (uint64_t)cnt * (uint64_t)orc_group_weight(S_row[j], smax);
+        total += W[j];
+    }
+    /* plain insertion sort: W descending, j ascending */
+    int nz = 0;
+    for (int j = 0; j < Ck; ++j) {
+        if (k_offsets[j + 1] - k_offsets[j] <= 0) continue;
+        int pos = nz++;
+        while (pos > 0) {
+            const int prev = order[pos - 1];
+            if (W[prev] > W[j] || (W[prev] == W[j] && prev < j)) break;
+            order[pos] = prev;
+            --pos;
+        }
+        order[pos] = j;
+    }
+    for (int r = 0; r < Ck; ++r) exact_groups[r] = -1;
+    uint64_t cum = 0;
+    int64_t keys = 0;
+    int n = 0;
+    for (int r = 0; r < nz; ++r) {
+        const int j = order[r];
+        exact_groups[n++] = j;
+        cum += W[j];
+        keys += k_offsets[j + 1] - k_offsets[j];
+        if (cum * 1048576ull >= (uint64_t)p_fix * total && keys >= floor_keys) break;
+    }
+    counts[0] = n;
+    counts[1] = (int32_t)keys;
+    counts[2] = 0;
+    if (W_out) memcpy(W_out, W, sizeof(uint64_t) * (size_t)Ck);
+    if (total_out) *total_out = total;
+    free(order); free(W);
+    return ORC_OK;
+}
+
+/* Whole head: scores from the given centroids, then every query group.      */
+int orc_select_top_p(const float* cq, int Cq, const float* ck, int Ck, int d, float scale,
+                     const int32_t* k_offsets, float top_p, int64_t floor_keys,
+                     int32_t* exact_groups, int32_t* counts)
+{
+    float* S = (float*)malloc(sizeof(float) * (size_t)Cq * (size_t)Ck);
+    if (!S) return ORC_ERR_NOMEM;
+    orc_scores(cq, Cq, ck, Ck, d, scale, S);
+    int rc = ORC_OK;
+    for (int i = 0; i < Cq && rc == ORC_OK; ++i)
+        rc = orc_select_top_p_group(S + (int64_t)i * Ck, k_offsets, Ck, top_p, floor_keys,
+                                    exact_groups + (int64_t)i * Ck, counts + 3 * i, NULL, NULL);
+    free(S);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Product-quantised per-query voting (the selection rule of the abstract:
  * queries and keys are product-quantised so that a block score is cheap for
  * every query, each query votes for its top blocks, and the cluster attends
