@@ -242,14 +242,15 @@ def job_time(t_total_ms, e2e_ms_per_call, steps, world, dist=None, device="cpu")
     return ms_call, ms_call / world, e2e_max / world
 
 
-def budget_point(ig, Q, K, V, w, exact, sample, D, dn, *, seed, layer, reps=3, ws=None):
+def budget_point(ig, Q, K, V, w, exact, sample, D, dn, *, seed, layer, reps=3, ws=None, **sel):
     """ms per instagen_forward call (CUDA events, one warm-up, median of
     `reps`) and the relative L2 error of its output against the dense output
     D (||D|| = dn) for one (exact, sample) budget on the given inputs; also
-    the attended density of the call."""
+    the attended density of the call.  ``sel``: selection keywords of
+    make_params (e.g. selection="top_p", top_p=0.9, key_floor=0.1)."""
     import torch
     p = ig.make_params(w.B, w.H, w.N, w.d, w.Cq, w.Ck, iters=w.iters, exact_frac=exact, sample_frac=sample,
-                       seed=seed, layer=layer)
+                       seed=seed, layer=layer, **sel)
     if ws is None or ws.numel() < ig.workspace_size(p):
         ws = torch.empty(ig.workspace_size(p), dtype=torch.uint8, device=Q.device)
     O = torch.empty_like(Q)
@@ -268,8 +269,28 @@ def budget_point(ig, Q, K, V, w, exact, sample, D, dn, *, seed, layer, reps=3, w
     cnt = it["counts"].long()
     qoff = it["q_offsets"].long()
     pairs = float(((qoff[..., 1:] - qoff[..., :-1]) * (cnt[..., 1] + cnt[..., 2])).sum())
-    return {"exact_frac": exact, "sample_frac": sample, "ms_per_call": round(statistics.median(ts), 3),
-            "rel_l2_vs_dense": round(err, 4), "density": round(pairs / (w.B * w.H * w.N * w.N), 4)}
+    out = {"exact_frac": exact, "sample_frac": sample, "ms_per_call": round(statistics.median(ts), 3),
+           "rel_l2_vs_dense": round(err, 4), "density": round(pairs / (w.B * w.H * w.N * w.N), 4)}
+    if sel:
+        out.update({k: v for k, v in sel.items()})
+        out.pop("exact_frac")
+        out.pop("sample_frac")
+    return out
+
+
+def top_p_comparator(ig, Q, K, V, w, D, dn, rank):
+    """The SVG2-style top-p selection (no sample; key floor 0.1) at p = 0.5,
+    0.75, 0.9, 0.95, each beside the importance-sampled call at the same
+    attended density (exact and sampled shares each half of that density):
+    ms per call and error against dense attention."""
+    rows = []
+    for tp in (0.5, 0.75, 0.9, 0.95):
+        a = budget_point(ig, Q, K, V, w, 0.0, 0.0, D, dn, seed=1000 + rank, layer=rank, selection="top_p",
+                         top_p=tp, key_floor=0.1)
+        half = round(a["density"] / 2, 4)
+        b = budget_point(ig, Q, K, V, w, half, half, D, dn, seed=1000 + rank, layer=rank)
+        rows.append({"top_p": a, "importance_at_matched_density": b})
+    return rows
 
 
 def stack_sample_sweep(ig, dev, args):
@@ -465,6 +486,7 @@ def main():
             extra["density_sweep"] = [budget_point(ig, Q, K, V, w, ex, sa, Df, dn, seed=1000 + rank, layer=rank,
                                                    ws=ws)
                                       for ex, sa in ((0.04, 0.04), (0.32, 0.32))]
+            extra["top_p_comparator"] = top_p_comparator(ig, Q, K, V, w, Df, dn, rank)
             del Df
         del D
 

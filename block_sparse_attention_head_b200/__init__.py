@@ -25,7 +25,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "_build", "libinstagen.so")
 
 IMPORTANCE, UNIFORM = 0, 1
-CENTROID, PQ_VOTE = 0, 1  # instagen_selection
+CENTROID, PQ_VOTE, TOP_P = 0, 1, 2  # instagen_selection
 
 
 class InstaGenError(RuntimeError):
@@ -38,7 +38,8 @@ class Params(ctypes.Structure):
                 ("Cq", ctypes.c_int32), ("Ck", ctypes.c_int32), ("kmeans_iters", ctypes.c_int32),
                 ("exact_frac", ctypes.c_float), ("sample_frac", ctypes.c_float),
                 ("softmax_scale", ctypes.c_float), ("seed", ctypes.c_uint64), ("layer", ctypes.c_uint32),
-                ("sampling", ctypes.c_int32), ("selection", ctypes.c_int32)]
+                ("sampling", ctypes.c_int32), ("selection", ctypes.c_int32), ("top_p", ctypes.c_float),
+                ("key_floor", ctypes.c_float)]
 
 
 class ForwardLayout(ctypes.Structure):
@@ -127,14 +128,18 @@ def _need(t: torch.Tensor, name: str, dtype, shape=None):
 
 def make_params(B: int, H: int, N: int, d: int, Cq: int, Ck: int, *, iters: int = 10, exact_frac: float = 0.16,
                 sample_frac: float = 0.16, softmax_scale: Optional[float] = None, seed: int = 0, layer: int = 0,
-                sampling: int | str = IMPORTANCE, selection: int | str = CENTROID) -> Params:
+                sampling: int | str = IMPORTANCE, selection: int | str = CENTROID, top_p: float = 0.9,
+                key_floor: float = 0.1) -> Params:
+    """``selection``: "centroid" (default), "pq_vote", or "top_p" (the comparator:
+    keep the key groups holding the share ``top_p`` of the estimated mass and at
+    least ``key_floor`` of the keys; no sample, so sample_frac must be 0)."""
     if isinstance(sampling, str):
         sampling = {"importance": IMPORTANCE, "uniform": UNIFORM}[sampling]
     if isinstance(selection, str):
-        selection = {"centroid": CENTROID, "pq_vote": PQ_VOTE}[selection]
+        selection = {"centroid": CENTROID, "pq_vote": PQ_VOTE, "top_p": TOP_P}[selection]
     scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
     return Params(B, H, N, d, Cq, Ck, iters, exact_frac, sample_frac, scale, seed & (2 ** 64 - 1), layer, sampling,
-                  selection)
+                  selection, top_p, key_floor)
 
 
 def exact_budget(p: Params) -> int:

@@ -36,9 +36,17 @@ int check_params(const instagen_params* p) {
     return IG_ERR_INVALID_ARG;
   if (!std::isfinite(p->softmax_scale) || !(p->softmax_scale > 0.f)) return IG_ERR_INVALID_ARG;
   if (p->sampling != IG_SAMPLE_IMPORTANCE && p->sampling != IG_SAMPLE_UNIFORM) return IG_ERR_INVALID_ARG;
-  if (p->selection != IG_SELECT_CENTROID && p->selection != IG_SELECT_PQ_VOTE) return IG_ERR_INVALID_ARG;
-  // votes enter the rank key saturated at 2^20 - 1: a group has fewer queries
-  if (p->selection == IG_SELECT_PQ_VOTE && p->N > 0xFFFFF) return IG_ERR_UNSUPPORTED;
+  if (p->selection != IG_SELECT_CENTROID && p->selection != IG_SELECT_PQ_VOTE && p->selection != IG_SELECT_TOP_P)
+    return IG_ERR_INVALID_ARG;
+  // votes enter the rank key saturated at 2^20 - 1: a group has fewer queries;
+  // top-p compares masses (< N * 2^24) scaled by 2^20 in 64 bits
+  if ((p->selection == IG_SELECT_PQ_VOTE || p->selection == IG_SELECT_TOP_P) && p->N > 0xFFFFF)
+    return IG_ERR_UNSUPPORTED;
+  if (p->selection == IG_SELECT_TOP_P) {
+    if (!(p->top_p >= 0.f && p->top_p <= 1.f) || !(p->key_floor >= 0.f && p->key_floor <= 1.f))
+      return IG_ERR_INVALID_ARG;
+    if (llround((double)p->sample_frac * (double)p->N) != 0) return IG_ERR_INVALID_ARG;  // no sample
+  }
   return IG_OK;
 }
 
@@ -184,6 +192,9 @@ int select_impl(const float* cq, const float* ck, const int32_t* k_offsets, cons
   a.mode = p->sampling;
   a.bh0 = bh0;
   a.votes = votes;
+  a.top_p = p->selection == IG_SELECT_TOP_P ? 1 : 0;
+  a.p_fix = llround((double)p->top_p * 1048576.0);
+  a.floor_keys = budget(p->key_floor, p->N);
   a.exact_groups = exact_groups;
   a.counts = counts;
   a.sample_pos = sample_pos;

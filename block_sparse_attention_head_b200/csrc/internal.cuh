@@ -62,6 +62,9 @@ struct SelectArgs {
   int mode;
   int bh0;  // global index of head 0 of this launch (the Philox counter's head)
   const int32_t* votes;  // [BH,Cq,Ck] product-quantised votes, or null (rank by S alone)
+  int top_p;             // 1: top-p selection (rank by mass, keep a share p_fix / 2^20, no sample)
+  long long p_fix;       // round(top_p * 2^20)
+  long long floor_keys;  // least number of kept keys
   int32_t* exact_groups;
   int32_t* counts;
   int32_t* sample_pos;

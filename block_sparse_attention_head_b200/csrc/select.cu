@@ -149,6 +149,81 @@ __global__ void __launch_bounds__(kSelThreads)
   }
   __syncthreads();
 
+  if (a.top_p) {
+    // Top-p selection (the comparator of the Figure 2 caption, SVG2-style):
+    // mass W_j = |K_j| q_j with the integer weights taken over every
+    // non-empty group, ranked by W descending (ties: lower j; rank key =
+    // (2^44 - 1 - W) << 12 | j), kept until the share of the total reaches
+    // p_fix / 2^20 and the kept keys reach floor_keys; no sample.
+    constexpr unsigned long long kMaxW = (1ull << 44) - 1;
+    for (int j = tid; j < Ck; j += kSelThreads)
+      if (koff[j + 1] > koff[j]) atomicMax(&s_smax_bits, float_order(S[j]));
+    if (tid == 0) s_nexact = 0x7fffffff;  // first rank that satisfies both conditions
+    __syncthreads();
+    const uint32_t ob_all = s_smax_bits;
+    const float smax_all = __uint_as_float((ob_all & 0x80000000u) ? (ob_all & 0x7fffffffu) : ~ob_all);
+    for (int j = tid; j < ck_pow2; j += kSelThreads) {
+      unsigned long long key = ~0ull;
+      if (j < Ck && koff[j + 1] > koff[j]) {
+        const unsigned long long W =
+            (unsigned long long)(koff[j + 1] - koff[j]) * group_weight(S[j], smax_all);
+        key = ((kMaxW - W) << 12) | (unsigned)j;
+      }
+      keys[j] = key;
+    }
+    __syncthreads();
+    for (int k = 2; k <= ck_pow2; k <<= 1) {
+      for (int jj = k >> 1; jj > 0; jj >>= 1) {
+        for (int x = tid; x < ck_pow2; x += kSelThreads) {
+          const int y = x ^ jj;
+          if (y > x) {
+            const unsigned long long u = keys[x], v = keys[y];
+            const bool up = (x & k) == 0;
+            if ((u > v) == up) {
+              keys[x] = v;
+              keys[y] = u;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    // cumulative mass (cdf) and kept keys (qinv as scratch) in rank order
+    for (int r = tid; r < Ck; r += kSelThreads) {
+      const unsigned long long key = keys[r];
+      const bool ne = key != ~0ull;
+      const int j = (int)(key & kKeyJ);
+      cdf[r] = ne ? kMaxW - (key >> 12) : 0ull;
+      qinv[r] = ne ? (unsigned long long)(koff[j + 1] - koff[j]) : 0ull;
+    }
+    __syncthreads();
+    block_incl_scan_u64(cdf, Ck, wtot);
+    block_incl_scan_u64(qinv, Ck, wtot);
+    const unsigned long long T = cdf[Ck - 1];
+    int nz_local = 0;
+    for (int r = tid; r < Ck; r += kSelThreads) {
+      if (keys[r] == ~0ull) continue;
+      ++nz_local;
+      if (cdf[r] * 1048576ull >= (unsigned long long)a.p_fix * T && qinv[r] >= (unsigned long long)a.floor_keys)
+        atomicMin(&s_nexact, r);
+    }
+    atomicAdd(&s_nskipped, nz_local);  // here: the number of non-empty groups
+    __syncthreads();
+    const int n_keep = s_nexact == 0x7fffffff ? s_nskipped : s_nexact + 1;
+    int32_t* ex_top = a.exact_groups + gi * Ck;
+    for (int r = tid; r < Ck; r += kSelThreads) ex_top[r] = r < n_keep ? (int32_t)(keys[r] & kKeyJ) : -1;
+    for (long long t = tid; t < a.m; t += kSelThreads) {
+      a.sample_pos[gi * a.m + t] = -1;
+      a.sample_bias[gi * a.m + t] = 0.0f;
+    }
+    if (tid == 0) {
+      a.counts[gi * 3 + 0] = n_keep;
+      a.counts[gi * 3 + 1] = n_keep > 0 ? (int32_t)qinv[n_keep - 1] : 0;
+      a.counts[gi * 3 + 2] = 0;
+    }
+    return;
+  }
+
   // rank the non-empty groups: S descending, j ascending (bitonic sort of
   // keys; j < 4096 sits in the low 12 bits).  With votes (product-quantised
   // voting) the votes, descending, come first (20 bits, saturated).

@@ -54,10 +54,20 @@ typedef enum {
 } instagen_status;
 
 typedef enum { IG_SAMPLE_IMPORTANCE = 0, IG_SAMPLE_UNIFORM = 1 } instagen_sampling;
-/* How the exact set is ranked: by centroid scores (Figure 3 (b)-(c)), or by
+/* How the exact set is ranked: by centroid scores (Figure 3 (b)-(c)), by
  * product-quantised per-query votes (the abstract's rule; see
- * instagen_pq_votes). */
-typedef enum { IG_SELECT_CENTROID = 0, IG_SELECT_PQ_VOTE = 1 } instagen_selection;
+ * instagen_pq_votes), or by the top-p rule of the comparator the pages set
+ * InstaGen against (thelatestinai.com paper page, Figure 2 caption: SVG2 at
+ * top-p 0.5 to 0.95 with key floor 0.1; ICLR listing abstract: top-p keeps
+ * the best blocks until a target share of the attention mass is reached and
+ * skips the rest).  Top-p: key group j's estimated mass is |K_j| q_j (the
+ * sampler's integer weights, taken over every non-empty group), groups are
+ * kept in descending mass order (ties: lower j) until their share of the
+ * total reaches top_p (compared in integers as cum * 2^20 >= round(top_p *
+ * 2^20) * total) and at least round(key_floor * N) keys are kept; the
+ * first-ranked group is always kept; there is no sample (sample_frac must
+ * give m = 0) and exact_frac is unused. */
+typedef enum { IG_SELECT_CENTROID = 0, IG_SELECT_PQ_VOTE = 1, IG_SELECT_TOP_P = 2 } instagen_selection;
 
 typedef struct {
   int32_t B, H, N, d;        /* shapes; d in {64, 128}; N >= 1                     */
@@ -69,7 +79,9 @@ typedef struct {
   uint64_t seed;             /* Philox key                                           */
   uint32_t layer;            /* Philox counter word 3 (one stream per layer)         */
   int32_t sampling;          /* instagen_sampling                                    */
-  int32_t selection;         /* instagen_selection (PQ voting needs N < 2^20)        */
+  int32_t selection;         /* instagen_selection (PQ voting, top-p: N < 2^20)     */
+  float top_p;               /* top-p selection: mass share in [0, 1]                */
+  float key_floor;           /* top-p selection: least share of keys kept, in [0, 1] */
 } instagen_params;
 
 /* E and m for these parameters: the share times N rounded to nearest, halves

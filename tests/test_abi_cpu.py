@@ -34,10 +34,11 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_params_struct_layout():
-    # instagen_params: 7 int32, 3 float, uint64 (8-aligned at 40), uint32, 2 int32
-    assert ctypes.sizeof(ig.Params) == 64
+    # instagen_params: 7 int32, 3 float, uint64 (8-aligned at 40), uint32, 2 int32, 2 float
+    assert ctypes.sizeof(ig.Params) == 72
     assert ig.Params.seed.offset == 40
     assert ig.Params.selection.offset == 56
+    assert ig.Params.top_p.offset == 60 and ig.Params.key_floor.offset == 64
     assert ctypes.sizeof(ig.ForwardLayout) == 18 * ctypes.sizeof(ctypes.c_size_t)
 
 
@@ -70,7 +71,7 @@ def test_workspace_layout(lib):
 
 @pytest.mark.parametrize("field,value,code", [
     ("d", 96, 2), ("d", 0, 2), ("N", 0, 1), ("B", 0, 1), ("Cq", 0, 1), ("Ck", 5000, 2),
-    ("sampling", 7, 1), ("exact_frac", -0.1, 1), ("sample_frac", float("nan"), 1),
+    ("sampling", 7, 1), ("exact_frac", -0.1, 1), ("sample_frac", float("nan"), 1), ("selection", 3, 1),
 ])
 def test_invalid_params_rejected_on_host(lib, field, value, code):
     p = ig.make_params(1, 2, 1000, 64, 8, 16)
@@ -138,3 +139,22 @@ def test_pq_vote_selection_checks_on_host(lib):
     p = ig.make_params(1, 40, 75600, 128, 100, 500, selection="pq_vote")
     # codebooks [40][2][16][16][8] fp32 + key-group codes [40][500][16]
     assert lib.instagen_pq_votes_workspace_size(ctypes.byref(p)) == 40 * 2 * 16 * 16 * 8 * 4 + 40 * 500 * 16
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(top_p=1.5), 1), (dict(top_p=-0.1), 1), (dict(key_floor=2.0), 1), (dict(top_p=float("nan")), 1),
+    (dict(sample_frac=0.01), 1), (dict(N=1 << 20), 2),
+])
+def test_top_p_params_rejected_on_host(lib, kw, code):
+    args = dict(N=1000, top_p=0.9, key_floor=0.1, sample_frac=0.0)
+    args.update(kw)
+    N = args.pop("N")
+    p = ig.make_params(1, 2, N, 64, 8, 16, selection="top_p", **args)
+    assert lib.instagen_workspace_size(ctypes.byref(p)) == 0
+    rc = lib.instagen_forward(None, None, None, None, ctypes.byref(p), None, 0, None)
+    assert rc == code
+
+
+def test_top_p_params_accepted(lib):
+    p = ig.make_params(1, 2, 75600, 128, 100, 500, selection="top_p", top_p=0.95, key_floor=0.1, sample_frac=0.0)
+    assert ig.workspace_size(p) > 0
