@@ -148,7 +148,9 @@ int instagen_cluster(const void* X, int32_t C, int32_t iters, const float* init,
  *   The array is held by every GPU that loads the library until the process
  *   exits.  The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture.
+ *   before any stream capture.  The address is looked up again when the
+ *   device's current context changes (after cudaDeviceReset, for instance),
+ *   so the first call after such a change must also come before any capture.
  *   All calls share the one array and it keeps the last call's contents;
  *   every element a call reads is written by the same call first, so nothing
  *   needs clearing, but calls that overlap on the GPU (other streams, other
