@@ -21,8 +21,10 @@
  *   - Tensors are contiguous, row-major, on the current CUDA device.
  *     Q, K, V, O: [B, H, N, d] bf16.  B and H are folded: head bh = b*H + h.
  *   - Device pointers unless stated.  The caller owns every buffer; the
- *     library never allocates, frees or synchronises (except
- *     instagen_device_status, which synchronises the given stream).
+ *     library never allocates or frees memory and never synchronises
+ *     (except instagen_device_status, which synchronises the given stream).
+ *     instagen_forward_host alone creates helper streams and events, and
+ *     releases them before it returns.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
  *     All work is enqueued asynchronously on it.
  *   - Return value: an instagen_status.  Argument errors are detected on the
