@@ -41,8 +41,8 @@
 // Warps: 0 TMEM owner and MMA warp of chain 0, 1 MMA warp of chain 1 (each
 // chain's MMAs come from one elected lane, in order; two issuers keep the
 // tensor pipe fed while either one waits on a barrier or sits in the issue of
-// an MMA instruction, which takes about as long as the MMA itself), 2-3
-// producer (cp.async 16-byte
+// an MMA instruction, which takes about as long as the MMA itself), 2-3 and
+// 12-13 producer, one warp per SM sub-partition (cp.async 16-byte
 // row gathers into the 128-byte-swizzled operand layout, completion tracked
 // by the stage mbarriers so the producer never blocks on memory; the key side
 // rows are plain shared stores), 4-11 softmax: warp w owns TMEM lane quarter
@@ -56,8 +56,8 @@
 namespace ig {
 
 namespace {
-constexpr int kAttnThreads = 384;
-constexpr int kProducers = 64;
+constexpr int kAttnThreads = 448;
+constexpr int kProducers = 128;
 constexpr int kSoftmaxThreads = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;
@@ -236,13 +236,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
 
   if (ntk < 1) {
     if (tid == 0) raise_error(kErrIndex);  // empty key list: nothing to attend
-  } else if (warp == 2 || warp == 3) {
+  } else if (warp == 2 || warp == 3 || warp >= 12) {
     // ================================================================ producer
-    const int tp = tid - 64;  // 0..63: rows tp and tp + 64 of every K/V tile
+    // four warps, one per SM sub-partition: producer warp pw owns rows
+    // [32 pw, 32 pw + 32) of every K/V tile, lane l row 32 pw + l
+    const int pw = warp < 4 ? warp - 2 : warp - 10;
+    const int tp = 32 * pw + lane;  // 0..127
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {  // query rows tp + 64h of the 256-row pair
-      const int r = tp + 64 * h;
-      const int t = r >> 7, rr = r & 127;
+    for (int h = 0; h < 2; ++h) {  // query rows tp and tp + 128 of the 256-row pair
+      const int r = tp + 128 * h;
+      const int t = h, rr = tp;
       bool valid = rr < (t == 0 ? rows0 : rows1);
       int tok = 0;
       if (valid) {
@@ -265,112 +268,94 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(AttnArgs a) 
     // two bf16 terms, so one more K=16 step of the S product adds the slot's
     // log-weight (and -inf for padding slots) to every score of its column.
     // Only the first 16 bytes of a key side row change per tile; this thread
-    // owns rows tp and tp + 64 of every side block.
+    // owns row tp of every side block.
     auto side_off = [](int r, int chunk) -> uint32_t {
       return (uint32_t)((r >> 3) * 256 + chunk * 128 + (r & 7) * 16);
     };
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int r = tp + 64 * h;
-      st_shared_v4(qx_s + side_off(r, 0), 0x3F803F80u, 0u, 0u, 0u);  // bf16 1.0, 1.0
-      st_shared_v4(qx_s + side_off(r, 1), 0u, 0u, 0u, 0u);
-      st_shared_v4(kx_s + side_off(r, 1), 0u, 0u, 0u, 0u);
-      st_shared_v4(kx_s + L::kSideBytes + side_off(r, 1), 0u, 0u, 0u, 0u);
-    }
+    st_shared_v4(qx_s + side_off(tp, 0), 0x3F803F80u, 0u, 0u, 0u);  // bf16 1.0, 1.0
+    st_shared_v4(qx_s + side_off(tp, 1), 0u, 0u, 0u, 0u);
+    st_shared_v4(kx_s + side_off(tp, 1), 0u, 0u, 0u, 0u);
+    st_shared_v4(kx_s + L::kSideBytes + side_off(tp, 1), 0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
     mbar_arrive(q_full);
     const float inv_scale = kLog2e / a.scale_log2;
     // slot log-weight over the scale: 0 for exact keys, -inf past the list
-    auto slot_w = [&](int j, int r) -> float {
-      const int l = j * 128 + r;
+    auto slot_w = [&](int j) -> float {
+      const int l = j * 128 + tp;
       if (l < Xi) return 0.f;
       if (l < Lk) return __ldg(sbias + (l - Xi)) * inv_scale;
       return -__int_as_float(0x7f800000);
     };
-    auto side_row = [&](uint32_t base, int r, float w) {
-      const float hi = __bfloat162float(__float2bfloat16_rn(w));
-      const float lo = isfinite(w) ? w - hi : 0.f;
-      st_shared_v4(base + side_off(r, 0), pack_bf16x2(hi, lo), 0u, 0u, 0u);
-    };
-    // Warp w of the producer owns rows [64w, 64w+64) of every K/V tile; lane l
-    // resolves the permuted key positions of rows 64w+l and 64w+32+l (one tile
-    // ahead, since sample positions come from global memory).  The copies are
-    // issued lane -> 16-byte chunk of a row, so one warp instruction moves
-    // whole 256-byte rows (full L2 sectors).
-    const int pw = tp >> 5;
-    // Slot -> permuted key position.  Each row stream of a lane visits
-    // increasing slots (one per tile), so its exact group e (the last with
-    // gpre[e] <= slot) is found by walking forward from the previous one,
-    // about one step per tile, instead of a binary search per slot.
-    auto key_pos = [&](int j, int r, int& e) -> int {  // -1: padding slot
-      const int l = j * 128 + r;                       // slot of tile row r in the key list
+    // Slot -> permuted key position.  A lane visits increasing slots (one
+    // per tile), so its exact group e (the last with gpre[e] <= slot) is
+    // found by walking forward from the previous one, about one step per
+    // tile, instead of a binary search per slot.
+    int e = 0;
+    auto key_pos = [&](int j) -> int {  // -1: padding slot
+      const int l = j * 128 + tp;
       if (l < Xi) {
         while (e + 1 < n_exact && gpre[e + 1] <= l) ++e;
         return gstart[e] + (l - gpre[e]);
       }
-      if (l < Lk) return __ldg(spos + (l - Xi));
-      return -1;
-    };
-    auto checked = [&](int p) -> int {
-      if (p >= N) {
-        raise_error(kErrIndex);
-        return -1;
+      if (l < Lk) {
+        const int p = __ldg(spos + (l - Xi));
+        if (p >= N) {
+          raise_error(kErrIndex);
+          return -1;
+        }
+        return p < 0 ? -1 : p;
       }
-      return p < 0 ? -1 : p;
+      return -1;
     };
     constexpr int kCpr = D / 8;       // 16-byte chunks per row
     constexpr int kRpi = 32 / kCpr;   // rows per warp instruction
+    constexpr int kIters = 32 / kRpi;
     const int rsub = lane / kCpr, ch = lane % kCpr;
-    // this lane's 16-byte chunk of rows i*kRpi + rsub (i = 0..64/kRpi-1) of the
-    // warp's 64 rows, from the row positions held by lanes (posA: rows 0-31,
-    // posB: rows 32-63)
     const uint32_t lane_dst = (uint32_t)((ch >> 3) * 16384);
-    // All row positions are fetched from their lanes first (independent
-    // shuffles, latencies overlapped), then the copies are issued back to
-    // back.
-    auto issue_rows = [&](const auto* base, uint32_t dst, int posA, int posB) {
-      const auto* head = base + (size_t)bh * N * D + ch * 8;
-      constexpr int kIters = 64 / kRpi;
-      int pr[kIters];
-#pragma unroll
-      for (int i = 0; i < kIters; ++i)
-        pr[i] = __shfl_sync(0xffffffffu, i * kRpi < 32 ? posA : posB, (i * kRpi + rsub) & 31);
+    // this lane's 16-byte chunk of rows 32 pw + i*kRpi + rsub of a tile; the
+    // row positions are fetched from their lanes once per tile and serve the
+    // K and the V copies; one warp instruction moves whole 256-byte rows
+    auto issue_rows = [&](const void* base, uint32_t dst, const int* pr) {
+      // 16-byte chunks: a row is D/8 of them
+      const uint4* head = reinterpret_cast<const uint4*>(base) + (size_t)bh * N * (D / 8) + ch;
 #pragma unroll
       for (int i = 0; i < kIters; ++i) {
-        const int r = 64 * pw + i * kRpi + rsub;
+        const int r = 32 * pw + i * kRpi + rsub;
         const int p = pr[i];
-        cp_async_16(dst + lane_dst + sw128_offset(r, ch & 7), head + (size_t)(p < 0 ? 0 : p) * D,
+        cp_async_16(dst + lane_dst + sw128_offset(r, ch & 7), head + (size_t)(p < 0 ? 0 : p) * (D / 8),
                     p < 0 ? 0u : 16u);
       }
     };
-    int eA = 0, eB = 0;  // exact-group cursors of the two row streams
-    const int rA = 64 * pw + lane, rB = 64 * pw + 32 + lane;
-    int nA = key_pos(0, rA, eA), nB = key_pos(0, rB, eB);
-    float wA = slot_w(0, rA), wB = slot_w(0, rB);
+    int npos = key_pos(0);
+    float nw = slot_w(0);
     for (int kt = 0; kt < ntk; ++kt) {
       const int s = kt & 1, use = kt >> 1;
-      const int posA = checked(nA), posB = checked(nB);
-      const float cwA = wA, cwB = wB;
+      const int pos = npos;
+      const float w = nw;
       if (kt + 1 < ntk) {
-        nA = key_pos(kt + 1, rA, eA);
-        nB = key_pos(kt + 1, rB, eB);
-        wA = slot_w(kt + 1, rA);
-        wB = slot_w(kt + 1, rB);
+        npos = key_pos(kt + 1);
+        nw = slot_w(kt + 1);
       }
-      // warp-uniform waits: every lane reaches the shuffles below together
+      int pr[kIters];
+#pragma unroll
+      for (int i = 0; i < kIters; ++i) pr[i] = __shfl_sync(0xffffffffu, pos, i * kRpi + rsub);
+      // warp-uniform waits: every lane reaches the copies together
       if (kt >= 2 && !mbar_wait_warp(&k_empty[s], (use - 1) & 1, abort_flag)) break;
-      side_row(kx_s + s * L::kSideBytes, rA, cwA);
-      side_row(kx_s + s * L::kSideBytes, rB, cwB);
+      {
+        const float hi = __bfloat162float(__float2bfloat16_rn(w));
+        const float lo = isfinite(w) ? w - hi : 0.f;
+        st_shared_v4(kx_s + s * L::kSideBytes + side_off(tp, 0), pack_bf16x2(hi, lo), 0u, 0u, 0u);
+      }
       fence_proxy_async_smem();
       mbar_arrive(&k_full[s]);
-      issue_rows(a.Kp, k_s + s * L::kTileBytes, posA, posB);
+      issue_rows(a.Kp, k_s + s * L::kTileBytes, pr);
       cp_async_arrive_noinc(&k_full[s]);
       if (kt >= 2 && !mbar_wait_warp(&v_empty[s], (use - 1) & 1, abort_flag)) break;
-      issue_rows(a.Vp, v_s + s * L::kTileBytes, posA, posB);
+      issue_rows(a.Vp, v_s + s * L::kTileBytes, pr);
       cp_async_arrive_noinc(&v_full[s]);
     }
     cp_async_wait_all();
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 12) {
     // ================================================================= softmax
     const int qd = warp & 3;               // TMEM lane quarter
     const int hf = (warp - 4) >> 2;        // column half of S and O
