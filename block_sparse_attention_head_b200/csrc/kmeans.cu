@@ -163,6 +163,16 @@ struct AssignSmem {
 };
 }  // namespace
 
+// Next 256-token unit of a pair's range: (head, unit within the head).  The
+// roles walk their units with this cursor rather than dividing a 64-bit unit
+// index per unit, a long dependent chain for the single issuing threads.
+__device__ __forceinline__ void next_unit(int& bh, int& pr, int uph) {
+  if (++pr == uph) {
+    pr = 0;
+    ++bh;
+  }
+}
+
 // Folds 16 distance columns into the running (best, best_j): dist =
 // ||c||^2 - 2 x.c with the norms `nw` (shared memory, same address in every
 // lane).  Argmin by a pairwise tree in which the right operand wins only when
@@ -231,6 +241,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   const long long u0 = total * pair / npairs;
   const int nunits = (int)(total * (pair + 1) / npairs - u0);
   if (nunits <= 0) return;  // the same for both CTAs of the pair
+  const int bh0 = (int)(u0 / uph), pr0 = (int)(u0 % uph);  // first unit
   const int nchunks = g.c_pad / g.chunk;
   const int half = g.chunk / 2;         // centroid rows per CTA per chunk
   const int kblocks = 2 * L::kXBlocks;  // hi blocks then lo blocks
@@ -279,14 +290,13 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     int st = 0;
     bool ok = true;
     int ep = -1, cur_bh = -1;  // resident: epoch = head
-    for (int i = 0; i < nunits && ok; ++i) {
-      const int bh = (int)((u0 + i) / uph);
+    for (int i = 0, bh = bh0, pr = pr0; i < nunits && ok; ++i, next_unit(bh, pr, uph)) {
       if (resident) {
         if (bh == cur_bh) continue;
         cur_bh = bh;
         ++ep;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (ep >= 1 && !mbar_wait_sleep(&c_empty[kb], (ep - 1) & 1, abort_flag)) {
+          if (ep >= 1 && !mbar_wait(&c_empty[kb], (ep - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -299,7 +309,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       for (int c = 0; c < nchunks && ok; ++c) {
         for (int kb = 0; kb < kblocks; ++kb, ++st) {
           const int s = st % kAssignStages;
-          if (st >= kAssignStages && !mbar_wait_sleep(&c_empty[s], ((st / kAssignStages) - 1) & 1, abort_flag)) {
+          if (st >= kAssignStages && !mbar_wait(&c_empty[s], ((st / kAssignStages) - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -312,11 +322,9 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   } else if (warp == 2 && lane == 0) {
     // --------------------------------------------- token producer (both)
     prefetch_tmap(&tmap_x);
-    for (int i = 0; i < nunits; ++i) {
+    for (int i = 0, bh = bh0, pr = pr0; i < nunits; ++i, next_unit(bh, pr, uph)) {
       const int buf = i % kAssignXBufs;
-      if (i >= kAssignXBufs && !mbar_wait_sleep(&x_empty[buf], ((i / kAssignXBufs) - 1) & 1, abort_flag)) break;
-      const long long q = u0 + i;
-      const int bh = (int)(q / uph), pr = (int)(q % uph);
+      if (i >= kAssignXBufs && !mbar_wait(&x_empty[buf], ((i / kAssignXBufs) - 1) & 1, abort_flag)) break;
       const int row = bh * g.N + pr * 256 + (int)rank * 128;
       if (rank == 0) mbar_arrive_expect_tx(&x_full[buf], 2 * L::kXTileBytes);
       const uint32_t bar = mapa_shared(smem_u32(&x_full[buf]), 0);
@@ -326,33 +334,37 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ------------------------------------------------------- MMA (leader)
     const uint32_t idesc = umma_idesc_bf16(256, g.chunk, false, false);
+    // descriptors formed once: an operand's descriptor is the base one plus
+    // its byte offset / 16 (the start-address field; no carry out of it, as
+    // shared-memory offsets stay below 256 KB)
+    const uint64_t adesc0 = umma_desc_sw128(x_base, 16, 1024);
+    const uint64_t bdesc0 = umma_desc_sw128(st_base, 16, 1024);
     int st = 0, gc = 0;  // stage counter, global chunk counter (TMEM buffer phases)
     bool ok = true;
     int ep = -1, cur_bh = -1;  // resident: epoch = head
-    for (int i = 0; i < nunits && ok; ++i) {
+    for (int i = 0, bh = bh0, pr = pr0; i < nunits && ok; ++i, next_unit(bh, pr, uph)) {
       const int buf = i % kAssignXBufs;
-      if (!mbar_wait_sleep(&x_full[buf], (i / kAssignXBufs) & 1, abort_flag)) break;
-      const uint32_t xb = x_base + buf * L::kXTileBytes;
+      if (!mbar_wait(&x_full[buf], (i / kAssignXBufs) & 1, abort_flag)) break;
+      const uint64_t xdesc = adesc0 + (uint64_t)((buf * L::kXTileBytes) >> 4);
       if (resident) {
-        const int bh = (int)((u0 + i) / uph);
-        const bool head_ends = i + 1 == nunits || (int)((u0 + i + 1) / uph) != bh;
+        const bool head_ends = i + 1 == nunits || pr + 1 == uph;
         const int b = gc & 1;
-        if (gc >= 2 && !mbar_wait_sleep(&t_empty[b], ((gc >> 1) - 1) & 1, abort_flag)) break;
+        if (gc >= 2 && !mbar_wait(&t_empty[b], ((gc >> 1) - 1) & 1, abort_flag)) break;
         if (bh != cur_bh) {
           cur_bh = bh;
           ++ep;
           for (int kb = 0; kb < kblocks && ok; ++kb)
-            if (!mbar_wait_sleep(&c_full[kb], ep & 1, abort_flag)) ok = false;
+            if (!mbar_wait(&c_full[kb], ep & 1, abort_flag)) ok = false;
           if (!ok) break;
         }
         tc_fence_after();
+#pragma unroll
         for (int kb = 0; kb < kblocks; ++kb) {
           const int xkb = kb % L::kXBlocks;
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t adesc = umma_desc_sw128(xb + xkb * 16384 + k * 32, 16, 1024);
-            const uint64_t bdesc = umma_desc_sw128(st_base + kb * L::kStageBytes + k * 32, 16, 1024);
-            umma_bf16_ss_pair(tmem + (uint32_t)(b * 256), adesc, bdesc, idesc, (kb | k) != 0);
-          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_bf16_ss_pair(tmem + (uint32_t)(b * 256), xdesc + (uint64_t)((xkb * 16384 + k * 32) >> 4),
+                              bdesc0 + (uint64_t)((kb * L::kStageBytes + k * 32) >> 4), idesc, (kb | k) != 0);
         }
         if (head_ends)
           for (int kb = 0; kb < kblocks; ++kb) umma_commit_pair_mc(&c_empty[kb], 3);
@@ -363,24 +375,24 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       }
       for (int c = 0; c < nchunks && ok; ++c, ++gc) {
         const int b = gc & 1;
-        if (gc >= 2 && !mbar_wait_sleep(&t_empty[b], ((gc >> 1) - 1) & 1, abort_flag)) {
+        if (gc >= 2 && !mbar_wait(&t_empty[b], ((gc >> 1) - 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         for (int kb = 0; kb < kblocks; ++kb, ++st) {
           const int s = st % kAssignStages;
-          if (!mbar_wait_sleep(&c_full[s], (st / kAssignStages) & 1, abort_flag)) {
+          if (!mbar_wait(&c_full[s], (st / kAssignStages) & 1, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const int xkb = kb % L::kXBlocks;
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t adesc = umma_desc_sw128(xb + xkb * 16384 + k * 32, 16, 1024);
-            const uint64_t bdesc = umma_desc_sw128(st_base + s * L::kStageBytes + k * 32, 16, 1024);
-            umma_bf16_ss_pair(tmem + (uint32_t)(b * 256), adesc, bdesc, idesc, (kb | k) != 0);
-          }
+          const uint64_t sdesc = bdesc0 + (uint64_t)((s * L::kStageBytes) >> 4);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_bf16_ss_pair(tmem + (uint32_t)(b * 256), xdesc + (uint64_t)((xkb * 16384 + k * 32) >> 4),
+                              sdesc + (uint64_t)((k * 32) >> 4), idesc, (kb | k) != 0);
           umma_commit_pair_mc(&c_empty[s], 3);
         }
         if (!ok) break;
@@ -406,9 +418,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     float4* nw = norms_s + ew * 32;
     int gc = 0, hm = 0;  // global chunk counter, half merges of this group
     bool ok = true;
-    for (int i = 0; i < nunits && ok; ++i) {
-      const long long q = u0 + i;
-      const int bh = (int)(q / uph), pr = (int)(q % uph);
+    for (int i = 0, bh = bh0, pr = pr0; i < nunits && ok; ++i, next_unit(bh, pr, uph)) {
       const float* nrm = norms + (size_t)bh * g.c_pad;
       float best = __int_as_float(0x7f800000);
       int best_j = 0;
@@ -421,7 +431,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         const float kInf = __int_as_float(0x7f800000);
         const float4 nl = (4 * lane < ncol) ? __ldg(reinterpret_cast<const float4*>(nrm + c * g.chunk + h0) + lane)
                                             : make_float4(kInf, kInf, kInf, kInf);
-        if (!mbar_wait_warp_sleep(&t_full[b], (gc >> 1) & 1, abort_flag)) {
+        if (!mbar_wait_warp(&t_full[b], (gc >> 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -459,14 +469,14 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       const int hs = grp * 2 + (hm & 1);
       float2* hslot = hmerge + hs * 128 + r;
       if (hf == 1) {
-        if (hm >= 2 && !mbar_wait_warp_sleep(&h_empty[hs], ((hm >> 1) - 1) & 1, abort_flag)) break;
+        if (hm >= 2 && !mbar_wait_warp(&h_empty[hs], ((hm >> 1) - 1) & 1, abort_flag)) break;
         *hslot = make_float2(best, __int_as_float(best_j));
         __syncwarp();
         if (lane == 0) mbar_arrive(&h_full[hs]);
         ++hm;
         continue;
       }
-      if (!mbar_wait_warp_sleep(&h_full[hs], (hm >> 1) & 1, abort_flag)) break;
+      if (!mbar_wait_warp(&h_full[hs], (hm >> 1) & 1, abort_flag)) break;
       {
         const float2 o = *hslot;
         const int oj = __float_as_int(o.y);
@@ -486,12 +496,12 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       // merge the two groups' minima of this unit (slot i & 1)
       float2* slot = merge + (i & 1) * 128 + r;
       if (grp == 1) {
-        if (i >= 2 && !mbar_wait_warp_sleep(&m_empty[i & 1], ((i >> 1) - 1) & 1, abort_flag)) break;
+        if (i >= 2 && !mbar_wait_warp(&m_empty[i & 1], ((i >> 1) - 1) & 1, abort_flag)) break;
         *slot = make_float2(best, __int_as_float(best_j));
         __syncwarp();
         if (lane == 0) mbar_arrive(&m_full[i & 1]);
       } else {
-        if (!mbar_wait_warp_sleep(&m_full[i & 1], (i >> 1) & 1, abort_flag)) break;
+        if (!mbar_wait_warp(&m_full[i & 1], (i >> 1) & 1, abort_flag)) break;
         const float2 o = *slot;
         const int oj = __float_as_int(o.y);
         const int jj = (o.x < best || (o.x == best && oj < best_j)) ? oj : best_j;

@@ -58,19 +58,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// try_wait that lets the thread sleep (up to ~0.1 ms, woken when the phase
-// completes) instead of spinning, leaving issue slots to working warps.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(100000u)
-      : "memory");
-  return ok != 0;
-}
 // Bounded wait.  Returns false when the CTA is aborting (someone timed out).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -94,24 +81,6 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, v
 }
 
 // mbar_wait / mbar_wait_warp for threads that may wait long: sleeps between polls.
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_timer_ns();
-  while (true) {
-    if (mbar_try_wait_sleep(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
-      *abort_flag = 1;
-      raise_error(kErrTimeout);
-      return false;
-    }
-  }
-}
-__device__ __forceinline__ bool mbar_wait_warp_sleep(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  const bool ok = mbar_wait_sleep(bar, parity, abort_flag);
-  return __all_sync(0xffffffffu, ok) != 0;
-}
-
 // Bounded wait that ignores the abort flag (used to drain in-flight work).
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   const unsigned long long t0 = global_timer_ns();
