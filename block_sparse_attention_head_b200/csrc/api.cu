@@ -112,7 +112,10 @@ int run_cluster(const void* X, int C, int iters, const float* init, const instag
   CUtensorMap tx, tc;
   int rc = make_tmap_bf16(&tx, X, (uint64_t)BH * p->N, (uint64_t)p->d, 128);
   if (rc) return rc;
-  rc = make_tmap_bf16(&tc, sc.cmma, (uint64_t)BH * g.c_pad, (uint64_t)2 * p->d, (uint32_t)(g.chunk / 2));
+  // centroid operand boxes: half a chunk per CTA, or (hi | lo along N) the
+  // whole chunk, hi columns in one CTA and lo in the other
+  rc = make_tmap_bf16(&tc, sc.cmma, (uint64_t)BH * g.c_pad, (uint64_t)2 * p->d,
+                      (uint32_t)(ig::kmeans_hilo_n(g) ? g.chunk : g.chunk / 2));
   if (rc) return rc;
   const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
   cudaError_t e = ig::launch_kmeans_init(g, Xb, init, cent, sc, s);

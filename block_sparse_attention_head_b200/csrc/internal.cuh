@@ -18,6 +18,11 @@ struct KmeansGeom {
   int c_pad;   // C rounded up to a multiple of chunk
 };
 KmeansGeom kmeans_geom(int BH, int N, int d, int C);
+// One resident chunk of at most 128 centroids: the assign MMA takes the hi
+// and lo operand halves side by side along N (N = 2 * chunk, K = d; one CTA of
+// the pair holds the hi rows, the other the lo rows) instead of one after
+// the other along K, which halves its MMA count.
+__host__ __device__ inline bool kmeans_hilo_n(const KmeansGeom& g) { return g.c_pad == g.chunk && g.chunk <= 128; }
 
 // Scratch of one clustering call, carved from one 256-byte aligned block:
 // the operand rows and norms above, fp32 partial sums of the clusters that

@@ -249,6 +249,11 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   // loaded once per head (an epoch) into stages 0..kblocks-1 instead of once
   // per unit, and the MMA issuer waits on it only when the head changes.
   const bool resident = nchunks == 1 && kblocks <= kAssignStages;
+  // hi | lo along N: the resident chunk takes d / 64 stages, the hi rows in
+  // the leader, the lo rows in the peer; TMEM column j is x.c_hi of centroid
+  // j, column chunk + j its x.c_lo
+  const bool hilo = resident && kmeans_hilo_n(g);
+  const int rkb = hilo ? L::kXBlocks : kblocks;  // resident stages
 
   if (tid == 0) {
     for (int s = 0; s < kAssignStages; ++s) {
@@ -295,14 +300,18 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         if (bh == cur_bh) continue;
         cur_bh = bh;
         ++ep;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = 0; kb < rkb; ++kb) {
           if (ep >= 1 && !mbar_wait(&c_empty[kb], (ep - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
-          if (rank == 0) mbar_arrive_expect_tx(&c_full[kb], 2 * half * 128);
-          tma_load_2d_pair(st_base + kb * L::kStageBytes, &tmap_c, kb * 64, bh * g.c_pad + (int)rank * half,
-                           mapa_shared(smem_u32(&c_full[kb]), 0));
+          if (rank == 0) mbar_arrive_expect_tx(&c_full[kb], 2 * (hilo ? g.chunk : half) * 128);
+          if (hilo)
+            tma_load_2d_pair(st_base + kb * L::kStageBytes, &tmap_c, (int)rank * g.d + kb * 64, bh * g.c_pad,
+                             mapa_shared(smem_u32(&c_full[kb]), 0));
+          else
+            tma_load_2d_pair(st_base + kb * L::kStageBytes, &tmap_c, kb * 64, bh * g.c_pad + (int)rank * half,
+                             mapa_shared(smem_u32(&c_full[kb]), 0));
         }
         continue;
       }
@@ -333,7 +342,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     }
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ------------------------------------------------------- MMA (leader)
-    const uint32_t idesc = umma_idesc_bf16(256, g.chunk, false, false);
+    const uint32_t idesc = umma_idesc_bf16(256, hilo ? 2 * g.chunk : g.chunk, false, false);
     // descriptors formed once: an operand's descriptor is the base one plus
     // its byte offset / 16 (the start-address field; no carry out of it, as
     // shared-memory offsets stay below 256 KB)
@@ -353,21 +362,30 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         if (bh != cur_bh) {
           cur_bh = bh;
           ++ep;
-          for (int kb = 0; kb < kblocks && ok; ++kb)
+          for (int kb = 0; kb < rkb && ok; ++kb)
             if (!mbar_wait(&c_full[kb], ep & 1, abort_flag)) ok = false;
           if (!ok) break;
         }
         tc_fence_after();
+        if (hilo) {
 #pragma unroll
-        for (int kb = 0; kb < kblocks; ++kb) {
-          const int xkb = kb % L::kXBlocks;
+          for (int kb = 0; kb < L::kXBlocks; ++kb)
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16_ss_pair(tmem + (uint32_t)(b * 256), xdesc + (uint64_t)((xkb * 16384 + k * 32) >> 4),
-                              bdesc0 + (uint64_t)((kb * L::kStageBytes + k * 32) >> 4), idesc, (kb | k) != 0);
+            for (int k = 0; k < 4; ++k)
+              umma_bf16_ss_pair(tmem + (uint32_t)(b * 256), xdesc + (uint64_t)((kb * 16384 + k * 32) >> 4),
+                                bdesc0 + (uint64_t)((kb * L::kStageBytes + k * 32) >> 4), idesc, (kb | k) != 0);
+        } else {
+#pragma unroll
+          for (int kb = 0; kb < kblocks; ++kb) {
+            const int xkb = kb % L::kXBlocks;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma_bf16_ss_pair(tmem + (uint32_t)(b * 256), xdesc + (uint64_t)((xkb * 16384 + k * 32) >> 4),
+                                bdesc0 + (uint64_t)((kb * L::kStageBytes + k * 32) >> 4), idesc, (kb | k) != 0);
+          }
         }
         if (head_ends)
-          for (int kb = 0; kb < kblocks; ++kb) umma_commit_pair_mc(&c_empty[kb], 3);
+          for (int kb = 0; kb < rkb; ++kb) umma_commit_pair_mc(&c_empty[kb], 3);
         umma_commit_pair_mc(&t_full[b], 3);
         ++gc;
         umma_commit_pair_mc(&x_empty[buf], 3);
@@ -440,11 +458,24 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         nw[lane] = nl;
         __syncwarp();
         const uint32_t col0 = tmem + lane_off + (uint32_t)(b * 256 + h0);
+        float va[16], vb[16];
+        if (hilo) {
+          // 16 centroids at a time: their hi and lo products, added
+          for (int cb = 0; cb < ncol; cb += 16) {
+            tmem_ld16(col0 + cb, va);
+            tmem_ld16(col0 + g.chunk + cb, vb);
+            tmem_wait_ld();
+            pin_regs16(va);
+            pin_regs16(vb);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) va[e] += vb[e];
+            assign_reduce16(va, nw + cb / 4, h0 + cb, best, best_j);
+          }
+        }
         // 16-column groups, the next group's TMEM load in flight while one is
         // reduced (each wait covers the one load then outstanding)
-        float va[16], vb[16];
-        if (ncol > 0) tmem_ld16(col0, va);
-        for (int cb = 0; cb < ncol; cb += 32) {
+        if (!hilo && ncol > 0) tmem_ld16(col0, va);
+        for (int cb = 0; cb < ncol && !hilo; cb += 32) {
           tmem_wait_ld();
           pin_regs16(va);
           if (cb + 16 < ncol) tmem_ld16(col0 + cb + 16, vb);
