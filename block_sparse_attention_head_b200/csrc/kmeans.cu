@@ -128,7 +128,7 @@ cudaError_t launch_kmeans_init(const KmeansGeom& g, const __nv_bfloat16* X, cons
 // here: M = 128 or N = 128 MMAs leave the tensor pipe half idle on issue and
 // shared-memory reads, while one M = 256, N = 256 MMA per K-step keeps it
 // busy.  Persistent: the pairs walk contiguous ranges of units over all
-// heads.  Token tiles are double-buffered (the next unit streams in from HBM
+// heads.  Token tiles are triple-buffered (the next units stream in from HBM
 // during the current one) and the centroid halves stream through a ring of
 // K-blocks of 64 columns (TMA, 128-byte swizzle).  TMEM: 2 buffers x 256 fp32
 // columns; epilogue group b reduces the chunks that land in buffer b, split
