@@ -196,6 +196,33 @@ def test_kmeans_one_step_matches_oracle(oracle_mod, oracle_runs, case):
     ig.device_status()
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("C", [40, 128, 150, 300, 600])
+def test_kmeans_assign_layouts_match_oracle(oracle_mod, C, d):
+    """Each operand layout of the assign kernel, one step from the oracle's
+    initial centroids: one resident chunk of <= 128 centroids (hi and lo
+    products side by side along N: C = 40, 128), one resident chunk above
+    128 (hi then lo along K: C = 150), and centroids streamed in two and three
+    chunks (C = 300, 600)."""
+    H, N = 2, 3001
+    Q, K, V = workloads.random_small(40 + C + d, N, d, n_centres=max(8, C // 4), sigma=0.3, H=H)
+    p = ig.make_params(1, H, N, d, C, C, iters=1)
+    Xn = [np_(K[0, h].float()) for h in range(H)]
+    init = np.stack([oracle_mod.kmeans_init(x, C) for x in Xn])[None]
+    cent, assign, perm, offs = ig.cluster(K.cuda(), C, 1, p, init=cuda(init))
+    ga, gc = np_(assign)[0], np_(cent)[0]
+    for h in range(H):
+        oa, _ = oracle_mod.kmeans_assign(Xn[h], init[0, h])
+        agree = np.mean(ga[h] == oa)
+        assert agree >= 0.999, f"C={C} d={d} head {h}: {agree}"
+        assert ga[h].min() >= 0 and ga[h].max() < C
+        x = Xn[h].astype(np.float64)
+        for j in np.unique(ga[h]):
+            np.testing.assert_allclose(gc[h, j], x[ga[h] == j].mean(0), rtol=0, atol=2e-4)
+        assert np.array_equal(np_(perm)[0, h], np.argsort(ga[h], kind="stable"))
+    ig.device_status()
+
+
 @pytest.mark.parametrize("iters", [1, 3])
 def test_kmeans_large_clusters(oracle_mod, iters):
     """Clusters of ~10k members, which the centroid update splits into pieces
