@@ -87,17 +87,20 @@ EncodeTiledFn encode_fn() {
 }
 
 // 2-D bf16 row-major [rows, cols] tensor, box {64 columns, box_rows rows},
-// 128-byte swizzle (the UMMA K-major SWIZZLE_128B layout), zero fill outside.
-int make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// 128-byte swizzle (the UMMA K-major SWIZZLE_128B layout), zero fill outside;
+// or (box_cols 16) box {16 columns, box_rows rows} with the 32-byte swizzle of
+// the UMMA K-major SWIZZLE_32B layout.
+int make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                   uint32_t box_cols = 64) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return IG_ERR_CUDA;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, box_cols == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? IG_OK : IG_ERR_CUDA;
 }
 
@@ -109,7 +112,7 @@ int run_cluster(const void* X, int C, int iters, const float* init, const instag
   if (!ws || ws_bytes < ig::kmeans_scratch_bytes(g) || (reinterpret_cast<uintptr_t>(ws) & 255u))
     return IG_ERR_WORKSPACE;
   const ig::KmeansScratch sc = ig::kmeans_scratch_carve(g, ws);
-  CUtensorMap tx, tc;
+  CUtensorMap tx, tc, tn;
   int rc = make_tmap_bf16(&tx, X, (uint64_t)BH * p->N, (uint64_t)p->d, 128);
   if (rc) return rc;
   // centroid operand boxes: half a chunk per CTA, or (hi | lo along N) the
@@ -117,10 +120,15 @@ int run_cluster(const void* X, int C, int iters, const float* init, const instag
   rc = make_tmap_bf16(&tc, sc.cmma, (uint64_t)BH * g.c_pad, (uint64_t)2 * p->d,
                       (uint32_t)(ig::kmeans_hilo_n(g) ? g.chunk : g.chunk / 2));
   if (rc) return rc;
+  // norm rows: the same rows per CTA, 16 columns (hi | lo: the lo CTA takes
+  // the zero columns 16-31)
+  rc = make_tmap_bf16(&tn, sc.nrow, (uint64_t)BH * g.c_pad, (uint64_t)ig::kNormCols,
+                      (uint32_t)(ig::kmeans_hilo_n(g) ? g.chunk : g.chunk / 2), 16);
+  if (rc) return rc;
   const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
   cudaError_t e = ig::launch_kmeans_init(g, Xb, init, cent, sc, s);
   for (int it = 0; it < iters && e == cudaSuccess; ++it) {
-    e = ig::launch_kmeans_assign(g, &tx, &tc, sc.norms, assign, s);
+    e = ig::launch_kmeans_assign(g, &tx, &tc, &tn, assign, s);
     if (e == cudaSuccess) e = ig::launch_count_sort(assign, BH, p->N, C, perm, offsets, s);
     if (e == cudaSuccess) e = ig::launch_kmeans_update(g, Xb, perm, offsets, cent, sc, s);
   }

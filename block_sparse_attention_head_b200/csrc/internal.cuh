@@ -11,7 +11,15 @@ namespace ig {
 // ----------------------------------------------------------------- k-means
 // Operand layout of the centroids for the tensor-core distance GEMM:
 // [BH, c_pad, 2d] bf16, columns [0,d) = bf16(c) ("hi"), [d,2d) =
-// bf16(c - hi) ("lo"); norms [BH, c_pad] fp32 = ||c||^2 of the fp32 centroid.
+// bf16(c - hi) ("lo"); norm rows [BH, c_pad, kNormCols] bf16: -||c||^2 / 4
+// of the fp32 centroid in three bf16 terms at columns 0-2 and again at 8-10,
+// zeros elsewhere (padding rows: -inf at columns 0 and 8).  One more K = 16
+// step of the distance MMA, against a block of ones at columns 0-2 and 8-10
+// of every token row, adds -||c||^2 / 2 to x.c; the copies in both 16-byte
+// halves keep that sum independent of where a swizzle puts the halves.
+// Columns 16-31 are zeros (the hi | lo layout below takes them as the lo
+// CTA's norm block).
+constexpr int kNormCols = 32;
 struct KmeansGeom {
   int BH, N, d, C;
   int chunk;   // centroids per MMA chunk (multiple of 16, <= 256)
@@ -25,13 +33,13 @@ KmeansGeom kmeans_geom(int BH, int N, int d, int C);
 __host__ __device__ inline bool kmeans_hilo_n(const KmeansGeom& g) { return g.c_pad == g.chunk && g.chunk <= 128; }
 
 // Scratch of one clustering call, carved from one 256-byte aligned block:
-// the operand rows and norms above, fp32 partial sums of the clusters that
+// the operand rows and norm rows above, fp32 partial sums of the clusters that
 // the update splits into several row pieces ([BH, part_slots, d]), and one
 // arrival counter per (head, cluster) ([BH, C] int32, zeroed by the init
 // kernel and returned to zero by the update that consumes it).
 struct KmeansScratch {
   __nv_bfloat16* cmma;
-  float* norms;
+  __nv_bfloat16* nrow;
   float* partial;
   int32_t* arrive;
 };
@@ -42,7 +50,7 @@ KmeansScratch kmeans_scratch_carve(const KmeansGeom& g, void* ws);
 cudaError_t launch_kmeans_init(const KmeansGeom& g, const __nv_bfloat16* X, const float* init, float* cent,
                                const KmeansScratch& sc, cudaStream_t s);
 cudaError_t launch_kmeans_assign(const KmeansGeom& g, const CUtensorMap* tmap_x, const CUtensorMap* tmap_c,
-                                 const float* norms, int32_t* assign, cudaStream_t s);
+                                 const CUtensorMap* tmap_n, int32_t* assign, cudaStream_t s);
 cudaError_t launch_kmeans_update(const KmeansGeom& g, const __nv_bfloat16* X, const int32_t* perm,
                                  const int32_t* offsets, float* cent, const KmeansScratch& sc, cudaStream_t s);
 

@@ -46,7 +46,7 @@ size_t a256(size_t b) { return (b + 255) / 256 * 256; }
 
 size_t kmeans_scratch_bytes(const KmeansGeom& g) {
   const size_t BH = (size_t)g.BH;
-  return a256(BH * g.c_pad * 2 * g.d * sizeof(__nv_bfloat16)) + a256(BH * g.c_pad * sizeof(float)) +
+  return a256(BH * g.c_pad * 2 * g.d * sizeof(__nv_bfloat16)) + a256(BH * g.c_pad * kNormCols * sizeof(__nv_bfloat16)) +
          a256(BH * kmeans_part_slots(g) * g.d * sizeof(float)) + a256(BH * g.C * sizeof(int32_t));
 }
 
@@ -56,16 +56,35 @@ KmeansScratch kmeans_scratch_carve(const KmeansGeom& g, void* ws) {
   KmeansScratch sc;
   sc.cmma = reinterpret_cast<__nv_bfloat16*>(b);
   b += a256(BH * g.c_pad * 2 * g.d * sizeof(__nv_bfloat16));
-  sc.norms = reinterpret_cast<float*>(b);
-  b += a256(BH * g.c_pad * sizeof(float));
+  sc.nrow = reinterpret_cast<__nv_bfloat16*>(b);
+  b += a256(BH * g.c_pad * kNormCols * sizeof(__nv_bfloat16));
   sc.partial = reinterpret_cast<float*>(b);
   b += a256(BH * kmeans_part_slots(g) * g.d * sizeof(float));
   sc.arrive = reinterpret_cast<int32_t*>(b);
   return sc;
 }
 
-// Writes the hi/lo bf16 operand row and ||c||^2 for centroid row `c` (one warp).
-__device__ __forceinline__ void write_operand_row(const float* c, int d, __nv_bfloat16* hi_lo, float* norm,
+// Lane `lane` (0-31) of a warp writes column `lane` of a centroid's norm row
+// for ||c||^2 = ss (every lane holds ss); an infinite ss makes a padding row.
+__device__ __forceinline__ void write_norm_row(float ss, __nv_bfloat16* nrow, int lane) {
+  const int k = lane & 15;
+  float t = 0.f;
+  if (lane < 16 && (k == 0 || k == 8) && isinf(ss)) {
+    t = -ss;
+  } else if (lane < 16 && isfinite(ss) && (k & 7) < 3) {
+    // -ss / 4 = t0 + t1 + t2, each rounded to bf16 in turn
+    const float v = -0.25f * ss;
+    const float t0 = __bfloat162float(__float2bfloat16_rn(v));
+    const float t1 = __bfloat162float(__float2bfloat16_rn(v - t0));
+    const float t2 = __bfloat162float(__float2bfloat16_rn((v - t0) - t1));
+    t = (k & 7) == 0 ? t0 : (k & 7) == 1 ? t1 : t2;
+  }
+  nrow[lane] = __float2bfloat16_rn(t);
+}
+
+// Writes the hi/lo bf16 operand row and the norm row for centroid row `c`
+// (one warp).
+__device__ __forceinline__ void write_operand_row(const float* c, int d, __nv_bfloat16* hi_lo, __nv_bfloat16* nrow,
                                                   int lane) {
   float ss = 0.f;
   for (int k = lane; k < d; k += 32) {
@@ -77,14 +96,14 @@ __device__ __forceinline__ void write_operand_row(const float* c, int d, __nv_bf
     ss = fmaf(v, v, ss);
   }
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if (lane == 0) *norm = ss;
+  write_norm_row(ss, nrow, lane);
 }
 
 // Initial centroids (given, or token floor(j*N/C)) and their operand rows.
 // One warp per (bh, padded centroid row).
 __global__ void kmeans_init_kernel(KmeansGeom g, const __nv_bfloat16* __restrict__ X, const float* __restrict__ init,
                                    float* __restrict__ cent, __nv_bfloat16* __restrict__ cmma,
-                                   float* __restrict__ norms, int32_t* __restrict__ arrive) {
+                                   __nv_bfloat16* __restrict__ nrows, int32_t* __restrict__ arrive) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int total = g.BH * g.c_pad;
@@ -92,9 +111,10 @@ __global__ void kmeans_init_kernel(KmeansGeom g, const __nv_bfloat16* __restrict
   const int bh = warp / g.c_pad, j = warp % g.c_pad;
   if (j < g.C && lane == 0) arrive[(size_t)bh * g.C + j] = 0;
   __nv_bfloat16* op = cmma + ((size_t)bh * g.c_pad + j) * 2 * g.d;
+  __nv_bfloat16* nr = nrows + ((size_t)bh * g.c_pad + j) * kNormCols;
   if (j >= g.C) {  // padding row: zero operand, infinite norm, never selected
     for (int k = lane; k < 2 * g.d; k += 32) op[k] = __float2bfloat16_rn(0.f);
-    if (lane == 0) norms[(size_t)bh * g.c_pad + j] = __int_as_float(0x7f800000);
+    write_norm_row(__int_as_float(0x7f800000), nr, lane);
     return;
   }
   float* c = cent + ((size_t)bh * g.C + j) * g.d;
@@ -107,7 +127,7 @@ __global__ void kmeans_init_kernel(KmeansGeom g, const __nv_bfloat16* __restrict
     for (int k = lane; k < g.d; k += 32) c[k] = __bfloat162float(src[k]);
   }
   __syncwarp();
-  write_operand_row(c, g.d, op, norms + (size_t)bh * g.c_pad + j, lane);
+  write_operand_row(c, g.d, op, nr, lane);
 }
 
 cudaError_t launch_kmeans_init(const KmeansGeom& g, const __nv_bfloat16* X, const float* init, float* cent,
@@ -115,7 +135,7 @@ cudaError_t launch_kmeans_init(const KmeansGeom& g, const __nv_bfloat16* X, cons
   const long long warps = (long long)g.BH * g.c_pad;
   const int threads = 256;
   const long long blocks = (warps * 32 + threads - 1) / threads;
-  kmeans_init_kernel<<<(unsigned)blocks, threads, 0, s>>>(g, X, init, cent, sc.cmma, sc.norms, sc.arrive);
+  kmeans_init_kernel<<<(unsigned)blocks, threads, 0, s>>>(g, X, init, cent, sc.cmma, sc.nrow, sc.arrive);
   return cudaGetLastError();
 }
 
@@ -135,8 +155,12 @@ cudaError_t launch_kmeans_init(const KmeansGeom& g, const __nv_bfloat16* X, cons
 // between two halves of 4 warps that take the lower and upper half of the
 // chunk's columns (16-column TMEM loads, the next in flight while one is
 // reduced): the reduction waits on TMEM loads, so twice the warps keep twice
-// the loads in flight.  A unit's partial minima merge through shared memory,
-// the upper half into the lower, then group 1 into group 0.  Warps: 0
+// the loads in flight.  One more K = 16 step of each chunk's MMA adds
+// -||c||^2 / 2 (a block of ones in shared memory against the chunk's norm rows,
+// both 32-byte swizzled), so TMEM holds x.c - ||c||^2 / 2 and the epilogue is
+// a bare argmax with no per-column norm.  A unit's partial maxima merge
+// through shared memory, the upper half into the lower, then group 1 into
+// group 0.  Warps: 0
 // centroid producer, 1 TMEM owner + MMA issuer (leader CTA), 2 token
 // producer, 4 + 8h + 4b + q: group b, half h, TMEM lane quarter q.
 namespace {
@@ -153,8 +177,9 @@ struct AssignSmem {
   static constexpr int kStages = kX + kAssignXBufs * kXTileBytes;
   static constexpr int kMerge = kStages + kAssignStages * kStageBytes;  // [2 slots][128] (distance, index)
   static constexpr int kHMerge = kMerge + 2 * 128 * 8;                  // [group][2 slots][128] (distance, index)
-  static constexpr int kNorms = kHMerge + 4 * 128 * 8;                  // [16 epilogue warps][128] fp32
-  static constexpr int kBars = kNorms + 16 * 128 * 4;
+  // ones block of the norm step: 128 rows x 32 B (1024-aligned)
+  static constexpr int kOnes = (kHMerge + 4 * 128 * 8 + 1023) / 1024 * 1024;
+  static constexpr int kBars = kOnes + 128 * 32;
   // c_full, c_empty [stages]; x_full, x_empty [x bufs]; t_full, t_empty, m_full, m_empty [2]; fin;
   // h_full, h_empty [group][2]
   static constexpr int kNumBars = 2 * kAssignStages + 2 * kAssignXBufs + 8 + 1 + 8;
@@ -173,36 +198,29 @@ __device__ __forceinline__ void next_unit(int& bh, int& pr, int uph) {
   }
 }
 
-// Folds 16 distance columns into the running (best, best_j): dist =
-// ||c||^2 - 2 x.c with the norms `nw` (shared memory, same address in every
-// lane).  Argmin by a pairwise tree in which the right operand wins only when
-// strictly smaller, and the running minimum is replaced only by a strictly
-// smaller one, so ties keep the lowest index; padding centroids have an
-// infinite norm and never win.
-__device__ __forceinline__ void assign_reduce16(const float (&x)[16], const float4* nw, int j0, float& best,
-                                                int& best_j) {
+// Folds 16 columns of x.c - ||c||^2 / 2 into the running (best, best_j): the
+// largest value is the smallest distance ||c||^2 - 2 x.c.  Argmax by a
+// pairwise tree in which the right operand wins only when strictly larger,
+// and the running maximum is replaced only by a strictly larger one, so ties
+// keep the lowest index; padding centroids hold -inf and never win.
+__device__ __forceinline__ void assign_argmax16(const float (&x)[16], int j0, float& best, int& best_j) {
   float m[8];
   int ix[8];
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const float4 n = nw[u];
-    const float a0 = fmaf(-2.f, x[4 * u], n.x), a1 = fmaf(-2.f, x[4 * u + 1], n.y);
-    const float a2 = fmaf(-2.f, x[4 * u + 2], n.z), a3 = fmaf(-2.f, x[4 * u + 3], n.w);
-    ix[2 * u] = a1 < a0 ? 4 * u + 1 : 4 * u;
-    m[2 * u] = fminf(a0, a1);
-    ix[2 * u + 1] = a3 < a2 ? 4 * u + 3 : 4 * u + 2;
-    m[2 * u + 1] = fminf(a2, a3);
+  for (int u = 0; u < 8; ++u) {
+    ix[u] = x[2 * u + 1] > x[2 * u] ? 2 * u + 1 : 2 * u;
+    m[u] = fmaxf(x[2 * u], x[2 * u + 1]);
   }
 #pragma unroll
   for (int w = 4; w >= 1; w >>= 1) {
 #pragma unroll
     for (int k = 0; k < w; ++k) {
-      const bool lt = m[2 * k + 1] < m[2 * k];
-      ix[k] = lt ? ix[2 * k + 1] : ix[2 * k];
-      m[k] = fminf(m[2 * k], m[2 * k + 1]);
+      const bool gt = m[2 * k + 1] > m[2 * k];
+      ix[k] = gt ? ix[2 * k + 1] : ix[2 * k];
+      m[k] = fmaxf(m[2 * k], m[2 * k + 1]);
     }
   }
-  if (m[0] < best) {
+  if (m[0] > best) {
     best = m[0];
     best_j = j0 + ix[0];
   }
@@ -211,7 +229,7 @@ __device__ __forceinline__ void assign_reduce16(const float (&x)[16], const floa
 template <int D>
 __global__ void __launch_bounds__(kAssignThreads, 1)
     kmeans_assign_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_c,
-                         KmeansGeom g, const float* __restrict__ norms, int32_t* __restrict__ assign) {
+                         const __grid_constant__ CUtensorMap tmap_n, KmeansGeom g, int32_t* __restrict__ assign) {
   using L = AssignSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -229,7 +247,6 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   uint64_t* h_empty = t_full + 13;  // [group * 2 + slot]
   float2* merge = reinterpret_cast<float2*>(smem + L::kMerge);
   float2* hmerge = reinterpret_cast<float2*>(smem + L::kHMerge);
-  float4* norms_s = reinterpret_cast<float4*>(smem + L::kNorms);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
@@ -282,6 +299,14 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     tmem_alloc_pair(tmem_holder, 512);
     tmem_relinquish_pair();
   }
+  if (warp >= 4 && warp < 8) {
+    // A operand of the norm step: bf16 ones at columns 0-2 and 8-10 of every
+    // token row (the same 16 bytes in both halves of the 32-byte row)
+    const uint32_t row = smem_u32(smem + L::kOnes) + (uint32_t)(tid - 128) * 32u;
+    st_shared_v4(row, 0x3F803F80u, 0x00003F80u, 0u, 0u);
+    st_shared_v4(row + 16, 0x3F803F80u, 0x00003F80u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   cluster_sync_all();  // barriers and TMEM of both CTAs ready before any cross-CTA traffic
   tc_fence_after();
@@ -300,31 +325,39 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         if (bh == cur_bh) continue;
         cur_bh = bh;
         ++ep;
-        for (int kb = 0; kb < rkb; ++kb) {
+        // stages 0..rkb-1 the operand K-blocks, stage rkb the norm rows
+        const int nr = hilo ? g.chunk : half;  // centroid rows per CTA
+        const int row0 = hilo ? bh * g.c_pad : bh * g.c_pad + (int)rank * half;
+        for (int kb = 0; kb <= rkb; ++kb) {
           if (ep >= 1 && !mbar_wait(&c_empty[kb], (ep - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
-          if (rank == 0) mbar_arrive_expect_tx(&c_full[kb], 2 * (hilo ? g.chunk : half) * 128);
-          if (hilo)
-            tma_load_2d_pair(st_base + kb * L::kStageBytes, &tmap_c, (int)rank * g.d + kb * 64, bh * g.c_pad,
-                             mapa_shared(smem_u32(&c_full[kb]), 0));
+          if (rank == 0) mbar_arrive_expect_tx(&c_full[kb], 2 * nr * (kb < rkb ? 128 : 32));
+          const uint32_t bar = mapa_shared(smem_u32(&c_full[kb]), 0);
+          if (kb == rkb)
+            tma_load_2d_pair(st_base + kb * L::kStageBytes, &tmap_n, hilo ? (int)rank * 16 : 0, row0, bar);
           else
-            tma_load_2d_pair(st_base + kb * L::kStageBytes, &tmap_c, kb * 64, bh * g.c_pad + (int)rank * half,
-                             mapa_shared(smem_u32(&c_full[kb]), 0));
+            tma_load_2d_pair(st_base + kb * L::kStageBytes, &tmap_c, hilo ? (int)rank * g.d + kb * 64 : kb * 64,
+                             row0, bar);
         }
         continue;
       }
       for (int c = 0; c < nchunks && ok; ++c) {
-        for (int kb = 0; kb < kblocks; ++kb, ++st) {
+        // the chunk's operand K-blocks, then its norm rows
+        for (int kb = 0; kb <= kblocks; ++kb, ++st) {
           const int s = st % kAssignStages;
           if (st >= kAssignStages && !mbar_wait(&c_empty[s], ((st / kAssignStages) - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
-          if (rank == 0) mbar_arrive_expect_tx(&c_full[s], 2 * half * 128);
-          tma_load_2d_pair(st_base + s * L::kStageBytes, &tmap_c, kb * 64,
-                           bh * g.c_pad + c * g.chunk + (int)rank * half, mapa_shared(smem_u32(&c_full[s]), 0));
+          if (rank == 0) mbar_arrive_expect_tx(&c_full[s], 2 * half * (kb < kblocks ? 128 : 32));
+          const int row0 = bh * g.c_pad + c * g.chunk + (int)rank * half;
+          const uint32_t bar = mapa_shared(smem_u32(&c_full[s]), 0);
+          if (kb == kblocks)
+            tma_load_2d_pair(st_base + s * L::kStageBytes, &tmap_n, 0, row0, bar);
+          else
+            tma_load_2d_pair(st_base + s * L::kStageBytes, &tmap_c, kb * 64, row0, bar);
         }
       }
     }
@@ -348,6 +381,9 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     // shared-memory offsets stay below 256 KB)
     const uint64_t adesc0 = umma_desc_sw128(x_base, 16, 1024);
     const uint64_t bdesc0 = umma_desc_sw128(st_base, 16, 1024);
+    // norm step: the ones block against a stage of norm rows
+    const uint64_t ones_desc = umma_desc_sw32(smem_u32(smem + L::kOnes));
+    const uint64_t ndesc0 = umma_desc_sw32(st_base);
     int st = 0, gc = 0;  // stage counter, global chunk counter (TMEM buffer phases)
     bool ok = true;
     int ep = -1, cur_bh = -1;  // resident: epoch = head
@@ -362,7 +398,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         if (bh != cur_bh) {
           cur_bh = bh;
           ++ep;
-          for (int kb = 0; kb < rkb && ok; ++kb)
+          for (int kb = 0; kb <= rkb && ok; ++kb)
             if (!mbar_wait(&c_full[kb], ep & 1, abort_flag)) ok = false;
           if (!ok) break;
         }
@@ -384,8 +420,10 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
                                 bdesc0 + (uint64_t)((kb * L::kStageBytes + k * 32) >> 4), idesc, (kb | k) != 0);
           }
         }
+        umma_bf16_ss_pair(tmem + (uint32_t)(b * 256), ones_desc,
+                          ndesc0 + (uint64_t)((rkb * L::kStageBytes) >> 4), idesc, 1u);
         if (head_ends)
-          for (int kb = 0; kb < rkb; ++kb) umma_commit_pair_mc(&c_empty[kb], 3);
+          for (int kb = 0; kb <= rkb; ++kb) umma_commit_pair_mc(&c_empty[kb], 3);
         umma_commit_pair_mc(&t_full[b], 3);
         ++gc;
         umma_commit_pair_mc(&x_empty[buf], 3);
@@ -414,6 +452,18 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           umma_commit_pair_mc(&c_empty[s], 3);
         }
         if (!ok) break;
+        {  // norm step
+          const int s = st % kAssignStages;
+          if (!mbar_wait(&c_full[s], (st / kAssignStages) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          umma_bf16_ss_pair(tmem + (uint32_t)(b * 256), ones_desc,
+                            ndesc0 + (uint64_t)((s * L::kStageBytes) >> 4), idesc, 1u);
+          umma_commit_pair_mc(&c_empty[s], 3);
+          ++st;
+        }
         umma_commit_pair_mc(&t_full[b], 3);
       }
       if (ok) umma_commit_pair_mc(&x_empty[buf], 3);
@@ -433,30 +483,19 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     const int hcols = (g.chunk / 2 + 15) / 16 * 16;
     const int h0 = hf * hcols, h1 = min(g.chunk, h0 + hcols);
     const int ncol = h1 - h0;
-    float4* nw = norms_s + ew * 32;
     int gc = 0, hm = 0;  // global chunk counter, half merges of this group
     bool ok = true;
     for (int i = 0, bh = bh0, pr = pr0; i < nunits && ok; ++i, next_unit(bh, pr, uph)) {
-      const float* nrm = norms + (size_t)bh * g.c_pad;
-      float best = __int_as_float(0x7f800000);
+      float best = -__int_as_float(0x7f800000);
       int best_j = 0;
       for (int c = 0; c < nchunks; ++c, ++gc) {
         const int b = gc & 1;
         if (b != grp) continue;
-        // ||c||^2 of this half, fetched before the wait and kept in this
-        // warp's shared-memory slice; padding centroids have an infinite norm
-        // and never win (an infinite distance never compares below `best`)
-        const float kInf = __int_as_float(0x7f800000);
-        const float4 nl = (4 * lane < ncol) ? __ldg(reinterpret_cast<const float4*>(nrm + c * g.chunk + h0) + lane)
-                                            : make_float4(kInf, kInf, kInf, kInf);
         if (!mbar_wait_warp(&t_full[b], (gc >> 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        __syncwarp();  // every lane is done with the previous chunk's norms
-        nw[lane] = nl;
-        __syncwarp();
         const uint32_t col0 = tmem + lane_off + (uint32_t)(b * 256 + h0);
         float va[16], vb[16];
         if (hilo) {
@@ -469,7 +508,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
             pin_regs16(vb);
 #pragma unroll
             for (int e = 0; e < 16; ++e) va[e] += vb[e];
-            assign_reduce16(va, nw + cb / 4, h0 + cb, best, best_j);
+            assign_argmax16(va, h0 + cb, best, best_j);
           }
         }
         // 16-column groups, the next group's TMEM load in flight while one is
@@ -479,12 +518,12 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           tmem_wait_ld();
           pin_regs16(va);
           if (cb + 16 < ncol) tmem_ld16(col0 + cb + 16, vb);
-          assign_reduce16(va, nw + cb / 4, c * g.chunk + h0 + cb, best, best_j);
+          assign_argmax16(va, c * g.chunk + h0 + cb, best, best_j);
           if (cb + 16 < ncol) {
             tmem_wait_ld();
             pin_regs16(vb);
             if (cb + 32 < ncol) tmem_ld16(col0 + cb + 32, va);
-            assign_reduce16(vb, nw + cb / 4 + 4, c * g.chunk + h0 + cb + 16, best, best_j);
+            assign_argmax16(vb, c * g.chunk + h0 + cb + 16, best, best_j);
           }
         }
         tc_fence_before();
@@ -493,10 +532,10 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       }
       if (!ok) break;
       // with one chunk per unit the units alternate between the groups and
-      // only the group that reduced this one holds its minimum
+      // only the group that reduced this one holds its maximum
       if (nchunks == 1 && (gc - 1) % 2 != grp) continue;
-      // the upper half hands its minimum to the lower half of the group; on
-      // equal distances the lower centroid index wins
+      // the upper half hands its maximum to the lower half of the group; on
+      // equal values the lower centroid index wins
       const int hs = grp * 2 + (hm & 1);
       float2* hslot = hmerge + hs * 128 + r;
       if (hf == 1) {
@@ -511,7 +550,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       {
         const float2 o = *hslot;
         const int oj = __float_as_int(o.y);
-        if (o.x < best || (o.x == best && oj < best_j)) {
+        if (o.x > best || (o.x == best && oj < best_j)) {
           best = o.x;
           best_j = oj;
         }
@@ -524,7 +563,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         if (tok < g.N) assign[(size_t)bh * g.N + tok] = best_j;
         continue;
       }
-      // merge the two groups' minima of this unit (slot i & 1)
+      // merge the two groups' maxima of this unit (slot i & 1)
       float2* slot = merge + (i & 1) * 128 + r;
       if (grp == 1) {
         if (i >= 2 && !mbar_wait_warp(&m_empty[i & 1], ((i >> 1) - 1) & 1, abort_flag)) break;
@@ -535,7 +574,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         if (!mbar_wait_warp(&m_full[i & 1], (i >> 1) & 1, abort_flag)) break;
         const float2 o = *slot;
         const int oj = __float_as_int(o.y);
-        const int jj = (o.x < best || (o.x == best && oj < best_j)) ? oj : best_j;
+        const int jj = (o.x > best || (o.x == best && oj < best_j)) ? oj : best_j;
         __syncwarp();
         if (lane == 0) mbar_arrive(&m_empty[i & 1]);
         const int tok = pr * 256 + (int)rank * 128 + r;
@@ -554,7 +593,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
 }
 
 cudaError_t launch_kmeans_assign(const KmeansGeom& g, const CUtensorMap* tmap_x, const CUtensorMap* tmap_c,
-                                 const float* norms, int32_t* assign, cudaStream_t s) {
+                                 const CUtensorMap* tmap_n, int32_t* assign, cudaStream_t s) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -578,13 +617,13 @@ cudaError_t launch_kmeans_assign(const KmeansGeom& g, const CUtensorMap* tmap_x,
     cudaError_t e = cudaFuncSetAttribute(kmeans_assign_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)cfg.dynamicSmemBytes);
     if (e != cudaSuccess) return e;
-    return cudaLaunchKernelEx(&cfg, kmeans_assign_kernel<128>, *tmap_x, *tmap_c, g, norms, assign);
+    return cudaLaunchKernelEx(&cfg, kmeans_assign_kernel<128>, *tmap_x, *tmap_c, *tmap_n, g, assign);
   }
   cfg.dynamicSmemBytes = AssignSmem<64>::bytes();
   cudaError_t e = cudaFuncSetAttribute(kmeans_assign_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)cfg.dynamicSmemBytes);
   if (e != cudaSuccess) return e;
-  return cudaLaunchKernelEx(&cfg, kmeans_assign_kernel<64>, *tmap_x, *tmap_c, g, norms, assign);
+  return cudaLaunchKernelEx(&cfg, kmeans_assign_kernel<64>, *tmap_x, *tmap_c, *tmap_n, g, assign);
 }
 
 // ------------------------------------------------------------------ update
@@ -610,7 +649,8 @@ template <int kUpdThreads>
 __global__ void __launch_bounds__(kUpdThreads)
     kmeans_update_kernel(KmeansGeom g, const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ perm,
                          const int32_t* __restrict__ offsets, float* __restrict__ cent,
-                         __nv_bfloat16* __restrict__ cmma, float* __restrict__ norms, float* __restrict__ partial,
+                         __nv_bfloat16* __restrict__ cmma, __nv_bfloat16* __restrict__ nrows,
+                         float* __restrict__ partial,
                          int32_t* __restrict__ arrive, int part_slots) {
   __shared__ __align__(16) uint4 ring[kUpdDepth][kUpdThreads];  // later the slot partial sums
   __shared__ int rows_s[kUpdRows];  // the piece's token indices
@@ -761,10 +801,10 @@ __global__ void __launch_bounds__(kUpdThreads)
   for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
   if (lane == 0) red[wid] = sq;
   __syncthreads();
-  if (tid == 0) {
+  if (wid == 0) {
     float tot = 0.f;
     for (int w = 0; w < (g.d + 31) / 32; ++w) tot += red[w];
-    norms[(size_t)bh * g.c_pad + c] = tot;
+    write_norm_row(tot, nrows + ((size_t)bh * g.c_pad + c) * kNormCols, lane);
   }
 }
 
@@ -777,10 +817,10 @@ cudaError_t launch_kmeans_update(const KmeansGeom& g, const __nv_bfloat16* X, co
   // CTAs keep more of those chains in flight per SM.
   dim3 grid(g.C + (g.N + kUpdRows - 1) / kUpdRows, g.BH);
   if ((long long)g.N < 512LL * g.C)
-    kmeans_update_kernel<128><<<grid, 128, 0, s>>>(g, X, perm, offsets, cent, sc.cmma, sc.norms, sc.partial,
+    kmeans_update_kernel<128><<<grid, 128, 0, s>>>(g, X, perm, offsets, cent, sc.cmma, sc.nrow, sc.partial,
                                                    sc.arrive, kmeans_part_slots(g));
   else
-    kmeans_update_kernel<256><<<grid, 256, 0, s>>>(g, X, perm, offsets, cent, sc.cmma, sc.norms, sc.partial,
+    kmeans_update_kernel<256><<<grid, 256, 0, s>>>(g, X, perm, offsets, cent, sc.cmma, sc.nrow, sc.partial,
                                                    sc.arrive, kmeans_part_slots(g));
   return cudaGetLastError();
 }

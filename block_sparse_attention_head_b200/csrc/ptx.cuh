@@ -365,6 +365,19 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// UMMA shared-memory descriptor for a 32-byte-swizzled K-major operand of one
+// K = 16 bf16 step (layout type 6 = SWIZZLE_32B): rows of 32 B, 8-row atoms
+// 256 B apart (SBO), LBO unused (1).
+__device__ __forceinline__ uint64_t umma_desc_sw32(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>(256u >> 4) << 32;
+  d |= 1ull << 46;
+  d |= 6ull << 61;
+  return d;
+}
+
 // Shared-memory matrix descriptor, no swizzle, K-major: the operand is tiled
 // in 8-row x 16-byte core matrices (128 contiguous bytes each); lbo = byte
 // distance between core matrices adjacent along K, sbo = between core matrices
