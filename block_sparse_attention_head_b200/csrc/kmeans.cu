@@ -5,9 +5,11 @@
 // One Lloyd iteration = assign (tensor cores) -> stable counting sort ->
 // deterministic per-cluster mean.  Distances: ||x - c||^2 = ||x||^2 + ||c||^2
 // - 2 x.c; ||x||^2 is common to a token's candidates, so the argmin runs over
-// ||c||^2 - 2 x.c.  x.c is one tcgen05 GEMM with K = 2d: the bf16 token row is
-// multiplied by the centroid split into bf16 hi and lo halves (hi + lo carries
-// ~16 mantissa bits of the fp32 centroid), accumulated in fp32 in TMEM.
+// ||c||^2 - 2 x.c, i.e. the argmax of x.c - ||c||^2 / 2.  x.c is one tcgen05
+// GEMM with K = 2d: the bf16 token row is multiplied by the centroid split
+// into bf16 hi and lo halves (hi + lo carries ~16 mantissa bits of the fp32
+// centroid), accumulated in fp32 in TMEM, and one more K = 16 step adds
+// -||c||^2 / 2 from the centroid's norm row.
 #include "internal.cuh"
 #include "ptx.cuh"
 

@@ -123,8 +123,9 @@ int instagen_device_status(void* stream);
  *   assign    [B,H,N] int32 out: cluster of every token (last iteration).
  *   perm      [B,H,N] int32 out; offsets [B,H,C+1] int32 out (see above).
  *   ws        >= instagen_cluster_workspace_size(p, C) bytes, 256-B aligned.
- * Distances are evaluated on the tensor cores as ||c||^2 - 2 x.c with the fp32
- * centroid split into two bf16 halves (hi + lo) and fp32 accumulation.
+ * Distances are evaluated on the tensor cores as ||c||^2 - 2 x.c (the argmax
+ * of x.c - ||c||^2 / 2) with the fp32 centroid split into two bf16 halves (hi +
+ * lo), ||c||^2 / 2 in three bf16 terms, and fp32 accumulation.
  */
 int instagen_cluster(const void* X, int32_t C, int32_t iters, const float* init, const instagen_params* p,
                      float* centroids, int32_t* assign, int32_t* perm, int32_t* offsets, void* ws,
