@@ -13,7 +13,7 @@
 namespace ig {
 
 // --------------------------------------------------------- counting sort
-// One thread-block cluster of S CTAs per head (S <= 8); CTA r owns the r-th
+// One thread-block cluster of S CTAs per head (S <= 16); CTA r owns the r-th
 // of S contiguous token ranges, and warp w of it a contiguous sub-range.
 // Phase 1 counts every warp's range per cluster; the CTA totals are exchanged
 // through distributed shared memory, giving every CTA the global cluster
@@ -23,13 +23,18 @@ namespace ig {
 // token index.  The first kSortRegs steps of a warp's range stay in registers
 // from phase 1 to phase 3 (all their loads in flight at once; the ordered walk
 // then waits on no memory); longer ranges read the rest again.  The sort is a
-// single launch and needs no global scratch.
-constexpr int kSortMaxCtas = 8;
+// single launch and needs no global scratch.  The ordered walk is a chain of
+// dependent steps per warp, so when every head's cluster fits the device at
+// once (few heads), a head is spread over 16 CTAs (a non-portable cluster
+// size) with 24 register-held steps and 4 CTAs per SM, which shortens each
+// warp's chain; otherwise over 8 CTAs with 40 steps and 3 CTAs per SM.
+constexpr int kSortMaxCtas = 16;
+constexpr int kSortPortableCtas = 8;
 constexpr int kSortUnroll = 4;
-constexpr int kSortRegs = 40;     // 32-token steps per warp held in registers
-constexpr int kSortMaxWarps = 8;   // 256 threads, 3 CTAs per SM: 55 heads of 8 CTAs in one wave
+constexpr int kSortMaxWarps = 8;   // 256 threads per CTA
 
-__global__ void __launch_bounds__(kSortMaxWarps * 32, 3)
+template <int kSortRegs, int kMinBlocks>  // 32-token steps per warp held in registers; CTAs per SM
+__global__ void __launch_bounds__(kSortMaxWarps * 32, kMinBlocks)
     count_sort_kernel(const int32_t* __restrict__ assign, int N, int C, int32_t* __restrict__ perm,
                                   int32_t* __restrict__ offsets) {
   extern __shared__ int sort_smem[];  // cnt [nwarps][C], ctot [C], before [C], base [C+1]
@@ -156,28 +161,41 @@ __global__ void __launch_bounds__(kSortMaxWarps * 32, 3)
 
 cudaError_t launch_count_sort(const int32_t* assign, int BH, int N, int C, int32_t* perm, int32_t* offsets,
                               cudaStream_t s) {
-  // one CTA per 4096 tokens of a head, up to a cluster of 8; as many warps
-  // (<= kSortMaxWarps) as fit 160 KB of per-warp counters
+  // one CTA per 4096 tokens of a head, up to a cluster of 8 (or 16, see
+  // above); as many warps (<= kSortMaxWarps) as fit 160 KB of per-warp counters
   int S = (N + 4095) / 4096;
   S = S < 1 ? 1 : (S > kSortMaxCtas ? kSortMaxCtas : S);
   int nwarps = (int)((160 * 1024) / ((size_t)C * 4));
   nwarps = nwarps < 1 ? 1 : (nwarps > kSortMaxWarps ? kSortMaxWarps : nwarps);
   const size_t sm = ((size_t)nwarps * C + 3 * (size_t)C + 1) * sizeof(int);
-  cudaError_t e = cudaFuncSetAttribute(count_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(S, BH);
   cfg.blockDim = dim3(nwarps * 32);
   cfg.dynamicSmemBytes = sm;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = S;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, count_sort_kernel, assign, N, C, perm, offsets);
+  if (S > kSortPortableCtas) {
+    auto* k16 = count_sort_kernel<24, 4>;
+    cfg.gridDim = dim3(S, BH);
+    attr[0].val.clusterDim.x = S;
+    int active = 0;
+    if (cudaFuncSetAttribute(k16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) == cudaSuccess &&
+        cudaFuncSetAttribute(k16, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+        cudaOccupancyMaxActiveClusters(&active, k16, &cfg) == cudaSuccess && active >= BH)
+      return cudaLaunchKernelEx(&cfg, k16, assign, N, C, perm, offsets);
+    cudaGetLastError();  // clear a refusal; the portable size follows
+    S = kSortPortableCtas;
+  }
+  auto* k8 = count_sort_kernel<40, 3>;
+  cudaError_t e = cudaFuncSetAttribute(k8, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  cfg.gridDim = dim3(S, BH);
+  attr[0].val.clusterDim.x = S;
+  return cudaLaunchKernelEx(&cfg, k8, assign, N, C, perm, offsets);
 }
 
 // ---------------------------------------------------------------- gather
