@@ -129,7 +129,8 @@ int run_cluster(const void* X, int C, int iters, const float* init, const instag
   cudaError_t e = ig::launch_kmeans_init(g, Xb, init, cent, sc, s);
   for (int it = 0; it < iters && e == cudaSuccess; ++it) {
     e = ig::launch_kmeans_assign(g, &tx, &tc, &tn, assign, s);
-    if (e == cudaSuccess) e = ig::launch_count_sort(assign, BH, p->N, C, perm, offsets, s);
+    if (e == cudaSuccess)
+      e = ig::launch_count_sort(assign, BH, p->N, C, perm, offsets, sc.pmap, ig::kmeans_update_grid(g), s);
     if (e == cudaSuccess) e = ig::launch_kmeans_update(g, Xb, perm, offsets, cent, sc, s);
   }
   return cuda_status(e);
@@ -371,7 +372,8 @@ int instagen_permutation(const int32_t* assign, int32_t C, const instagen_params
   if ((rc = check_clusters(C))) return rc;
   if (!assign || !perm || !offsets) return IG_ERR_INVALID_ARG;
   return cuda_status(
-      ig::launch_count_sort(assign, p->B * p->H, p->N, C, perm, offsets, static_cast<cudaStream_t>(stream)));
+      ig::launch_count_sort(assign, p->B * p->H, p->N, C, perm, offsets, nullptr, 0,
+                            static_cast<cudaStream_t>(stream)));
 }
 
 int instagen_gather(const void* X, const int32_t* perm, const instagen_params* p, void* Xp, int32_t to_f16,

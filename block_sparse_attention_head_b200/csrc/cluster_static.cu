@@ -3,7 +3,7 @@
 // allocate device memory (see include/instagen.h).
 //
 // The scratch is the centroid operand of the distance GEMM ([BH, C_pad, 2d]
-// bf16), the norm rows ([BH, C_pad, 32] bf16), the update's partial sums and
+// bf16), the norm rows ([BH, C_pad, 32] bf16), the update's piece map, partial sums and
 // its arrival counters, the same layout instagen_cluster carves from a
 // caller-provided workspace.  Every element the kernels read from it is first
 // written by the same call (the init kernel writes every operand row, padding

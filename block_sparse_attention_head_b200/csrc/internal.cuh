@@ -32,14 +32,26 @@ KmeansGeom kmeans_geom(int BH, int N, int d, int C);
 // the other along K, which halves its MMA count.
 __host__ __device__ inline bool kmeans_hilo_n(const KmeansGeom& g) { return g.c_pad == g.chunk && g.chunk <= 128; }
 
+// The centroid update splits a cluster of n members into pieces of at most
+// kUpdRows consecutive permuted rows (an empty cluster is one empty piece);
+// its grid has kmeans_update_grid(g) CTAs per head, piece t of a head being
+// entry t of the head's piece map, {cluster, piece, pieces of the cluster,
+// first partial-sum slot of the cluster} ({-1, ...} past the last piece),
+// which the counting sort of the same iteration writes.
+constexpr int kUpdRows = 2048;
+__host__ __device__ inline int update_pieces(int n) { return n <= kUpdRows ? 1 : (n + kUpdRows - 1) / kUpdRows; }
+inline int kmeans_update_grid(const KmeansGeom& g) { return g.C + (g.N + kUpdRows - 1) / kUpdRows; }
+
 // Scratch of one clustering call, carved from one 256-byte aligned block:
-// the operand rows and norm rows above, fp32 partial sums of the clusters that
+// the operand rows and norm rows above, the piece map above ([BH,
+// kmeans_update_grid] int4), fp32 partial sums of the clusters that
 // the update splits into several row pieces ([BH, part_slots, d]), and one
 // arrival counter per (head, cluster) ([BH, C] int32, zeroed by the init
 // kernel and returned to zero by the update that consumes it).
 struct KmeansScratch {
   __nv_bfloat16* cmma;
   __nv_bfloat16* nrow;
+  int4* pmap;
   float* partial;
   int32_t* arrive;
 };
@@ -55,8 +67,10 @@ cudaError_t launch_kmeans_update(const KmeansGeom& g, const __nv_bfloat16* X, co
                                  const int32_t* offsets, float* cent, const KmeansScratch& sc, cudaStream_t s);
 
 // ------------------------------------------------------- permutation/gather
+// pmap (may be null): the centroid update's piece map, written from the
+// cluster sizes (kmeans_update_grid(geometry) entries per head).
 cudaError_t launch_count_sort(const int32_t* assign, int BH, int N, int C, int32_t* perm, int32_t* offsets,
-                              cudaStream_t s);
+                              int4* pmap, int pgrid, cudaStream_t s);
 // Up to two tensors gathered with the same permutation (X1 may be null); a
 // tensor with its f16 flag set is converted bf16 -> fp16.
 cudaError_t launch_gather_rows(const __nv_bfloat16* X0, const __nv_bfloat16* X1, const int32_t* perm, int BH,

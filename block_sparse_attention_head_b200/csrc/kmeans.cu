@@ -32,10 +32,6 @@ KmeansGeom kmeans_geom(int BH, int N, int d, int C) {
   return g;
 }
 
-// Rows summed by one CTA of the update; clusters with more members are split
-// into pieces of this many rows (in permuted order) whose partial sums are
-// added in piece order.
-constexpr int kUpdRows = 2048;
 
 // Partial-sum slots per head: the pieces of every cluster larger than one
 // piece.  A cluster of n > R rows has ceil(n/R) < 2n/R pieces, so all of them
@@ -49,6 +45,7 @@ size_t a256(size_t b) { return (b + 255) / 256 * 256; }
 size_t kmeans_scratch_bytes(const KmeansGeom& g) {
   const size_t BH = (size_t)g.BH;
   return a256(BH * g.c_pad * 2 * g.d * sizeof(__nv_bfloat16)) + a256(BH * g.c_pad * kNormCols * sizeof(__nv_bfloat16)) +
+         a256(BH * kmeans_update_grid(g) * sizeof(int4)) +
          a256(BH * kmeans_part_slots(g) * g.d * sizeof(float)) + a256(BH * g.C * sizeof(int32_t));
 }
 
@@ -60,6 +57,8 @@ KmeansScratch kmeans_scratch_carve(const KmeansGeom& g, void* ws) {
   b += a256(BH * g.c_pad * 2 * g.d * sizeof(__nv_bfloat16));
   sc.nrow = reinterpret_cast<__nv_bfloat16*>(b);
   b += a256(BH * g.c_pad * kNormCols * sizeof(__nv_bfloat16));
+  sc.pmap = reinterpret_cast<int4*>(b);
+  b += a256(BH * kmeans_update_grid(g) * sizeof(int4));
   sc.partial = reinterpret_cast<float*>(b);
   b += a256(BH * kmeans_part_slots(g) * g.d * sizeof(float));
   sc.arrive = reinterpret_cast<int32_t*>(b);
@@ -645,67 +644,28 @@ cudaError_t launch_kmeans_assign(const KmeansGeom& g, const CUtensorMap* tmap_x,
 // so the ring needs no barrier, only cp.async.wait_group.
 constexpr int kUpdDepth = 8;  // rows in flight per slot
 
-__device__ __forceinline__ int update_pieces(int n) { return n <= kUpdRows ? 1 : (n + kUpdRows - 1) / kUpdRows; }
 
 template <int kUpdThreads>
 __global__ void __launch_bounds__(kUpdThreads)
     kmeans_update_kernel(KmeansGeom g, const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ perm,
                          const int32_t* __restrict__ offsets, float* __restrict__ cent,
                          __nv_bfloat16* __restrict__ cmma, __nv_bfloat16* __restrict__ nrows,
-                         float* __restrict__ partial,
-                         int32_t* __restrict__ arrive, int part_slots) {
+                         float* __restrict__ partial, int32_t* __restrict__ arrive,
+                         const int4* __restrict__ pmap, int part_slots) {
   __shared__ __align__(16) uint4 ring[kUpdDepth][kUpdThreads];  // later the slot partial sums
   __shared__ int rows_s[kUpdRows];  // the piece's token indices
   __shared__ float red[32];
-  __shared__ int scan_np[kUpdThreads / 32], scan_mp[kUpdThreads / 32];
   __shared__ int s_c, s_piece, s_np, s_base, s_last;
   const int bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int32_t* off = offsets + (size_t)bh * (g.C + 1);
 
-  // (cluster, piece) of this CTA: exclusive scans over the clusters of the
-  // piece count and of the pieces that belong to multi-piece clusters
-  const int per = (g.C + kUpdThreads - 1) / kUpdThreads;
-  const int c0 = min(tid * per, g.C), c1 = min(c0 + per, g.C);
-  int np_own = 0, mp_own = 0;
-  for (int c = c0; c < c1; ++c) {
-    const int k = update_pieces(max(off[c + 1] - off[c], 0));
-    np_own += k;
-    if (k > 1) mp_own += k;
-  }
-  int np_inc = np_own, mp_inc = mp_own;
-  for (int o = 1; o < 32; o <<= 1) {
-    const int a = __shfl_up_sync(0xffffffffu, np_inc, o);
-    const int b = __shfl_up_sync(0xffffffffu, mp_inc, o);
-    if (lane >= o) {
-      np_inc += a;
-      mp_inc += b;
-    }
-  }
-  if (lane == 31) {
-    scan_np[wid] = np_inc;
-    scan_mp[wid] = mp_inc;
-  }
-  if (tid == 0) s_c = -1;
-  __syncthreads();
-  int at = np_inc - np_own, mb = mp_inc - mp_own;
-  for (int w = 0; w < wid; ++w) {
-    at += scan_np[w];
-    mb += scan_mp[w];
-  }
-  const int t = blockIdx.x;
-  if (t >= at && t < at + np_own) {
-    for (int c = c0; c < c1; ++c) {
-      const int k = update_pieces(max(off[c + 1] - off[c], 0));
-      if (t < at + k) {
-        s_c = c;
-        s_piece = t - at;
-        s_np = k;
-        s_base = mb;
-        break;
-      }
-      at += k;
-      if (k > 1) mb += k;
-    }
+  // (cluster, piece) of this CTA: entry blockIdx.x of the head's piece map
+  if (tid == 0) {
+    const int4 e = pmap[(size_t)bh * gridDim.x + blockIdx.x];
+    s_c = e.x;
+    s_piece = e.y;
+    s_np = e.z;
+    s_base = e.w;
   }
   __syncthreads();
   const int c = s_c;
@@ -817,13 +777,13 @@ cudaError_t launch_kmeans_update(const KmeansGeom& g, const __nv_bfloat16* X, co
   // few hundred rows take 128 threads: a CTA's time is then mostly the
   // latency of its dependent loads (offsets, permutation, rows), and smaller
   // CTAs keep more of those chains in flight per SM.
-  dim3 grid(g.C + (g.N + kUpdRows - 1) / kUpdRows, g.BH);
+  dim3 grid(kmeans_update_grid(g), g.BH);
   if ((long long)g.N < 512LL * g.C)
     kmeans_update_kernel<128><<<grid, 128, 0, s>>>(g, X, perm, offsets, cent, sc.cmma, sc.nrow, sc.partial,
-                                                   sc.arrive, kmeans_part_slots(g));
+                                                   sc.arrive, sc.pmap, kmeans_part_slots(g));
   else
     kmeans_update_kernel<256><<<grid, 256, 0, s>>>(g, X, perm, offsets, cent, sc.cmma, sc.nrow, sc.partial,
-                                                   sc.arrive, kmeans_part_slots(g));
+                                                   sc.arrive, sc.pmap, kmeans_part_slots(g));
   return cudaGetLastError();
 }
 

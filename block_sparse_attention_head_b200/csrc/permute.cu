@@ -36,7 +36,7 @@ constexpr int kSortMaxWarps = 8;   // 256 threads per CTA
 template <int kSortRegs, int kMinBlocks>  // 32-token steps per warp held in registers; CTAs per SM
 __global__ void __launch_bounds__(kSortMaxWarps * 32, kMinBlocks)
     count_sort_kernel(const int32_t* __restrict__ assign, int N, int C, int32_t* __restrict__ perm,
-                                  int32_t* __restrict__ offsets) {
+                                  int32_t* __restrict__ offsets, int4* __restrict__ pmap, int pgrid) {
   extern __shared__ int sort_smem[];  // cnt [nwarps][C], ctot [C], before [C], base [C+1]
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
@@ -157,10 +157,55 @@ __global__ void __launch_bounds__(kSortMaxWarps * 32, kMinBlocks)
     nxt = (i + 32 < s1) ? a[i + 32] : -1;  // next step's load in flight
     place(c, i);
   }
+  if (pmap != nullptr && r == 0) {
+    // The centroid update's piece map of this head, from the cluster sizes:
+    // exclusive prefixes over the clusters of their piece counts and of the
+    // pieces of multi-piece clusters (block-wide: a range of clusters per
+    // thread, warp scans, then the warp totals in order).
+    __shared__ int s_scan[2 * kSortMaxWarps];
+    const int nthr = blockDim.x;
+    const int per = (C + nthr - 1) / nthr;
+    const int c0 = min((int)threadIdx.x * per, C), c1 = min(c0 + per, C);
+    int np = 0, mp = 0;
+    for (int c = c0; c < c1; ++c) {
+      const int k = update_pieces(base[c + 1] - base[c]);
+      np += k;
+      if (k > 1) mp += k;
+    }
+    int npi = np, mpi = mp;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, npi, o), y = __shfl_up_sync(0xffffffffu, mpi, o);
+      if (lane >= o) {
+        npi += x;
+        mpi += y;
+      }
+    }
+    if (lane == 31) {
+      s_scan[warp] = npi;
+      s_scan[kSortMaxWarps + warp] = mpi;
+    }
+    __syncthreads();
+    int p0 = npi - np, m0 = mpi - mp, total = 0;
+    for (int w = 0; w < nwarps; ++w) {
+      if (w < warp) {
+        p0 += s_scan[w];
+        m0 += s_scan[kSortMaxWarps + w];
+      }
+      total += s_scan[w];
+    }
+    int4* pm = pmap + (size_t)bh * pgrid;
+    for (int c = c0; c < c1; ++c) {
+      const int k = update_pieces(base[c + 1] - base[c]);
+      for (int q = 0; q < k && p0 + q < pgrid; ++q) pm[p0 + q] = make_int4(c, q, k, m0);
+      p0 += k;
+      if (k > 1) m0 += k;
+    }
+    for (int t = total + (int)threadIdx.x; t < pgrid; t += nthr) pm[t] = make_int4(-1, 0, 0, 0);
+  }
 }
 
 cudaError_t launch_count_sort(const int32_t* assign, int BH, int N, int C, int32_t* perm, int32_t* offsets,
-                              cudaStream_t s) {
+                              int4* pmap, int pgrid, cudaStream_t s) {
   // one CTA per 4096 tokens of a head, up to a cluster of 8 (or 16, see
   // above); as many warps (<= kSortMaxWarps) as fit 160 KB of per-warp counters
   int S = (N + 4095) / 4096;
@@ -186,7 +231,7 @@ cudaError_t launch_count_sort(const int32_t* assign, int BH, int N, int C, int32
     if (cudaFuncSetAttribute(k16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) == cudaSuccess &&
         cudaFuncSetAttribute(k16, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
         cudaOccupancyMaxActiveClusters(&active, k16, &cfg) == cudaSuccess && active >= BH)
-      return cudaLaunchKernelEx(&cfg, k16, assign, N, C, perm, offsets);
+      return cudaLaunchKernelEx(&cfg, k16, assign, N, C, perm, offsets, pmap, pgrid);
     cudaGetLastError();  // clear a refusal; the portable size follows
     S = kSortPortableCtas;
   }
@@ -195,7 +240,7 @@ cudaError_t launch_count_sort(const int32_t* assign, int BH, int N, int C, int32
   if (e != cudaSuccess) return e;
   cfg.gridDim = dim3(S, BH);
   attr[0].val.clusterDim.x = S;
-  return cudaLaunchKernelEx(&cfg, k8, assign, N, C, perm, offsets);
+  return cudaLaunchKernelEx(&cfg, k8, assign, N, C, perm, offsets, pmap, pgrid);
 }
 
 // ---------------------------------------------------------------- gather

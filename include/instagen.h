@@ -133,7 +133,8 @@ int instagen_cluster(const void* X, int32_t C, int32_t iters, const float* init,
 
 /*
  * instagen_cluster without a workspace argument: the same k-means +
- * permutation, with its scratch (centroid operand and norm rows, partial sums
+ * permutation, with its scratch (centroid operand and norm rows, the update's
+ * piece map, partial sums
  * and arrival counters of the centroid update) in a device
  * array of INSTAGEN_CLUSTER_STATIC_SCRATCH_BYTES that the library itself
  * owns.  No counterpart on the method's pages; this exists for callers that
@@ -146,7 +147,7 @@ int instagen_cluster(const void* X, int32_t C, int32_t iters, const float* init,
  *   Scratch needed = instagen_cluster_workspace_size(p, C); larger requests
  *   return IG_ERR_WORKSPACE before anything is enqueued.  The scratch grows
  *   with B*H, C and d, and a little with N (8*d bytes per 2048 tokens of a
- *   head): 16 MiB covers up to 50 heads at C <= 512, d = 128, N = 75600
+ *   head): 16 MiB covers up to 48 heads at C <= 512, d = 128, N = 75600
  *   (e.g. the 40-head key clustering of Wan2.1-14B at 720p).
  *   The array is held by every GPU that loads the library until the process
  *   exits.  The first call on a device looks up the array's device address
