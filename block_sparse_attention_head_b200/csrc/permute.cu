@@ -25,8 +25,8 @@ namespace ig {
 // then waits on no memory); longer ranges read the rest again.  The sort is a
 // single launch and needs no global scratch.  The ordered walk is a chain of
 // dependent steps per warp, so when every head's cluster fits the device at
-// once (few heads), a head is spread over 16 CTAs (a non-portable cluster
-// size) with 24 register-held steps and 4 CTAs per SM, which shortens each
+// once, a head is spread over 16 or else 12 CTAs (non-portable cluster sizes)
+// with 24 or 32 register-held steps and 4 CTAs per SM, which shortens each
 // warp's chain; otherwise over 8 CTAs with 40 steps and 3 CTAs per SM.
 constexpr int kSortMaxCtas = 16;
 constexpr int kSortPortableCtas = 8;
@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(kSortMaxWarps * 32, kMinBlocks)
 
 cudaError_t launch_count_sort(const int32_t* assign, int BH, int N, int C, int32_t* perm, int32_t* offsets,
                               int4* pmap, int pgrid, cudaStream_t s) {
-  // one CTA per 4096 tokens of a head, up to a cluster of 8 (or 16, see
+  // one CTA per 4096 tokens of a head, up to a cluster of 8 (or 12 or 16, see
   // above); as many warps (<= kSortMaxWarps) as fit 160 KB of per-warp counters
   int S = (N + 4095) / 4096;
   S = S < 1 ? 1 : (S > kSortMaxCtas ? kSortMaxCtas : S);
@@ -223,18 +223,22 @@ cudaError_t launch_count_sort(const int32_t* assign, int BH, int N, int C, int32
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (S > kSortPortableCtas) {
-    auto* k16 = count_sort_kernel<24, 4>;
-    cfg.gridDim = dim3(S, BH);
-    attr[0].val.clusterDim.x = S;
+  // the largest of 16 and 12 CTAs per head whose clusters all fit the device
+  // at once, with enough register-held steps for a warp's range
+  for (int Sx = kSortMaxCtas; Sx > kSortPortableCtas && S > kSortPortableCtas; Sx -= 4) {
+    const int Su = S < Sx ? S : Sx;
+    const int steps = (int)(((long long)N + (long long)Su * nwarps * 32 - 1) / ((long long)Su * nwarps * 32)) + 1;
+    auto* kx = steps <= 24 ? count_sort_kernel<24, 4> : count_sort_kernel<32, 4>;
+    cfg.gridDim = dim3(Su, BH);
+    attr[0].val.clusterDim.x = Su;
     int active = 0;
-    if (cudaFuncSetAttribute(k16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) == cudaSuccess &&
-        cudaFuncSetAttribute(k16, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
-        cudaOccupancyMaxActiveClusters(&active, k16, &cfg) == cudaSuccess && active >= BH)
-      return cudaLaunchKernelEx(&cfg, k16, assign, N, C, perm, offsets, pmap, pgrid);
-    cudaGetLastError();  // clear a refusal; the portable size follows
-    S = kSortPortableCtas;
+    if (cudaFuncSetAttribute(kx, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) == cudaSuccess &&
+        cudaFuncSetAttribute(kx, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+        cudaOccupancyMaxActiveClusters(&active, kx, &cfg) == cudaSuccess && active >= BH && steps <= 32)
+      return cudaLaunchKernelEx(&cfg, kx, assign, N, C, perm, offsets, pmap, pgrid);
+    cudaGetLastError();  // clear a refusal; a smaller size follows
   }
+  S = S > kSortPortableCtas ? kSortPortableCtas : S;
   auto* k8 = count_sort_kernel<40, 3>;
   cudaError_t e = cudaFuncSetAttribute(k8, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
